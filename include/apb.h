@@ -1,0 +1,144 @@
+/*
+ * apb.h -- C ABI of the APB per-host prefill path on one B200 (sm_100a).
+ *
+ * Method: "APB: Accelerating Distributed Long-Context Inference by Passing
+ * Compressed Context Blocks across GPUs" (arXiv 2502.12085).  The juejin.cn
+ * post on APB, sections "APB 的主要功能" (main features) and "APB 的技术原理"
+ * (technical principles), states the steps implemented here:
+ *   - the sequence is split evenly into H context blocks (hosts); each host's
+ *     block is preceded by an anchor block, the start of the sequence, with
+ *     the query embedded at its start;
+ *   - each host compresses its KV with retaining heads and keeps the
+ *     important KV pairs (apb_score_compress);
+ *   - the compressed blocks are all-gathered and each host builds a passing
+ *     block from the blocks of the hosts before it (apb_build_passing); on one
+ *     GPU the H hosts are virtual and the all-gather is a local gather;
+ *   - each host attends over anchor + passing + its local block, and the
+ *     passing block is discarded afterwards (apb_block_attention).
+ *
+ * Conventions for every call:
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the
+ *     library allocates no device memory and keeps no state between calls
+ *     other than a per-process cache of driver entry points.
+ *   - Layouts are contiguous and token-major (row-major, last index fastest):
+ *       q      [N, Hq,  d]   bf16      (N = n_hosts * block_len)
+ *       k, v   [N, Hkv, d]   bf16
+ *       out    [N, Hq,  d]   bf16
+ *     Every tensor pointer must be 16-byte aligned.
+ *   - q head j uses kv head j / (Hq / Hkv) (consecutive grouping).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise, except apb_device_status.
+ *   - Arguments are checked on the host before anything is launched; a bad
+ *     argument returns APB_ERR_INVALID_ARG (or APB_ERR_UNSUPPORTED for a
+ *     valid but unimplemented shape) and launches nothing.  A failed launch
+ *     returns APB_ERR_CUDA.  Nothing aborts or throws across this boundary.
+ *   - Kernels that wait on on-chip barriers bound every wait; a wait that
+ *     runs out records APB_ERR_TIMEOUT in the workspace status word, the
+ *     kernel releases what it holds and returns, and apb_device_status
+ *     reports it.
+ */
+#ifndef APB_H_
+#define APB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  APB_OK = 0,
+  APB_ERR_INVALID_ARG = 1,
+  APB_ERR_UNSUPPORTED = 2,
+  APB_ERR_CUDA = 3,
+  APB_ERR_TIMEOUT = 4
+} apb_status;
+
+/* Sizes of one prefill.  Constraints (else APB_ERR_INVALID_ARG):
+ *   n_hosts >= 1, block_len >= 1, 0 <= query_len <= anchor_len <= block_len,
+ *   0 <= keep <= block_len, n_q_heads % n_kv_heads == 0.
+ * head_dim must be 64 or 128 and mlp_hidden 256 (else APB_ERR_UNSUPPORTED).
+ * softmax_scale <= 0 selects 1/sqrt(head_dim).  query_len only documents
+ * where the query segment sits (rows [0, query_len) of the anchor); no
+ * kernel treats those rows differently. */
+typedef struct apb_config {
+  int32_t n_hosts;      /* H */
+  int32_t block_len;    /* n: tokens per host */
+  int32_t anchor_len;   /* A: anchor rows [0, A), seen by hosts 1..H-1 */
+  int32_t query_len;    /* q_len */
+  int32_t keep;         /* top-k per (host, kv head) */
+  int32_t n_q_heads;    /* Hq */
+  int32_t n_kv_heads;   /* Hkv */
+  int32_t head_dim;     /* d */
+  int32_t mlp_hidden;   /* retaining-head hidden width */
+  float softmax_scale;
+} apb_config;
+
+/* Bytes of device workspace that apb_score_compress and apb_block_attention
+ * need: a 256-byte status block, plus Hkv*N*4 bytes (rounded up to 256) for
+ * the scores when apb_score_compress is given scores == NULL.  Returns 0 for
+ * a NULL or invalid config.  The caller zero-fills a workspace once before
+ * its first use (the status block must start at zero). */
+size_t apb_workspace_bytes(const apb_config* cfg);
+
+/* Step 1 (main features: KV compression with retaining heads; technical
+ * principles: the compressed block holds the important KV pairs).
+ * For every token t and kv head g the retaining-head stand-in computes
+ *     x = [k[t,g] ; v[t,g] ; mean_{j: j/G == g} q[t,j]]            (3d)
+ *     s[g,t] = w2[g] . SiLU(W1[g] x + b1[g]) + b2[g]
+ * in fp32, then keeps, for every host h and kv head g, the `keep` positions
+ * of [h*n, h*n+n) with the largest s (ties: the lower position wins).
+ *   w1 [Hkv, hidden, 3d], b1 [Hkv, hidden], w2 [Hkv, hidden], b2 [Hkv]: fp32
+ *   scores [Hkv, N] fp32 (out, may be NULL: then held in the workspace)
+ *   idx [H, Hkv, keep] int32 (out): global positions, ascending per (h, g)
+ *   workspace/ws_bytes: at least apb_workspace_bytes(cfg) bytes. */
+apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* k,
+                              const void* v, const float* w1, const float* b1,
+                              const float* w2, const float* b2, float* scores,
+                              int32_t* idx, void* workspace, size_t ws_bytes,
+                              void* stream);
+
+/* Step 2 (main features: communication; the all-gather of compressed blocks
+ * and the passing block built from the preceding hosts' blocks).
+ *   pass_k[g, h*keep + r, :] = k[idx[h, g, r], g, :]   (and likewise v)
+ *   pass_k, pass_v [Hkv, H*keep, d] bf16 (out), copied bit-exactly.
+ * Host h's passing block is rows [0, h*keep) of this layout.  An index
+ * outside [0, N) yields a zero row instead of a read. */
+apb_status apb_build_passing(const apb_config* cfg, const void* k, const void* v,
+                             const int32_t* idx, void* pass_k, void* pass_v,
+                             void* stream);
+
+/* Step 3 (main features: computation over anchor, passing and local block;
+ * the passing block is not kept afterwards).  For host h, local row i
+ * (t = h*n + i) and q head j (g = j / G):
+ *     keys = k[0:A, g] (only if h >= 1) ++ pass_k[g, 0:h*keep]
+ *            ++ k[h*n : t+1, g]
+ *     out[t, j] = softmax(q[t, j] . keys^T * scale) @ values
+ * bf16 tensor-core products, fp32 accumulation and online softmax.
+ *   out [N, Hq, d] bf16 (out); lse [Hq, N] fp32 natural log-sum-exp of the
+ *   scaled logits (out, may be NULL).
+ *   workspace/ws_bytes: at least 256 bytes (status block). */
+apb_status apb_block_attention(const apb_config* cfg, const void* q, const void* k,
+                               const void* v, const void* pass_k, const void* pass_v,
+                               void* out, float* lse, void* workspace, size_t ws_bytes,
+                               void* stream);
+
+/* Synchronises `stream`, then reads the status block of `workspace`:
+ * APB_ERR_TIMEOUT if a kernel recorded a bounded wait that ran out since the
+ * block was last cleared, else APB_OK (APB_ERR_CUDA if the reads fail).
+ * clear != 0 resets the block to zero afterwards. */
+apb_status apb_device_status(void* workspace, void* stream, int clear);
+
+/* Static, NUL-terminated name of a status code. */
+const char* apb_status_string(apb_status status);
+
+/* Human-readable detail of the last failure returned on the calling thread
+ * (static storage, valid until the next call on that thread). */
+const char* apb_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* APB_H_ */

@@ -1,0 +1,231 @@
+"""Python binding of the C ABI in include/apb.h (argument marshalling only).
+
+Every step of the path runs in the CUDA kernels of ``libapb.so``; this module
+checks tensor devices, dtypes and shapes, allocates outputs with torch when
+the caller gives none, and passes raw device pointers plus the current torch
+stream.  Importing it fails loudly when the in-tree library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libapb.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "apb.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m long_context_sparse_apb_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+APB_OK, APB_ERR_INVALID_ARG, APB_ERR_UNSUPPORTED, APB_ERR_CUDA, APB_ERR_TIMEOUT = range(5)
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("n_hosts", ctypes.c_int32), ("block_len", ctypes.c_int32),
+                ("anchor_len", ctypes.c_int32), ("query_len", ctypes.c_int32),
+                ("keep", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("mlp_hidden", ctypes.c_int32), ("softmax_scale", ctypes.c_float)]
+
+
+_P = ctypes.c_void_p
+_lib.apb_workspace_bytes.argtypes = [ctypes.POINTER(Config)]
+_lib.apb_workspace_bytes.restype = ctypes.c_size_t
+_lib.apb_score_compress.argtypes = [ctypes.POINTER(Config)] + [_P] * 10 + [ctypes.c_size_t, _P]
+_lib.apb_score_compress.restype = ctypes.c_int
+_lib.apb_build_passing.argtypes = [ctypes.POINTER(Config)] + [_P] * 6
+_lib.apb_build_passing.restype = ctypes.c_int
+_lib.apb_block_attention.argtypes = [ctypes.POINTER(Config)] + [_P] * 8 + [ctypes.c_size_t, _P]
+_lib.apb_block_attention.restype = ctypes.c_int
+_lib.apb_device_status.argtypes = [_P, _P, ctypes.c_int]
+_lib.apb_device_status.restype = ctypes.c_int
+_lib.apb_status_string.argtypes = [ctypes.c_int]
+_lib.apb_status_string.restype = ctypes.c_char_p
+_lib.apb_last_error.argtypes = []
+_lib.apb_last_error.restype = ctypes.c_char_p
+
+
+class APBError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = _lib.apb_status_string(status).decode()
+        detail = _lib.apb_last_error().decode()
+        super().__init__(f"{where}: {name}: {detail}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != APB_OK:
+        raise APBError(status, where)
+
+
+def status_string(status: int) -> str:
+    return _lib.apb_status_string(status).decode()
+
+
+def declared_symbols() -> list:
+    """Entry points declared in include/apb.h."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"\b(apb_[a-z_]+)\s*\(", text)))
+
+
+def make_config(cfg=None, **kw) -> Config:
+    """apb_config from an ``inputs.APBConfig`` (or keyword fields)."""
+    f = {}
+    if cfg is not None:
+        f = dict(n_hosts=cfg.n_hosts, block_len=cfg.block_len, anchor_len=cfg.anchor_len,
+                 query_len=cfg.query_len, keep=cfg.keep, n_q_heads=cfg.n_q_heads,
+                 n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, mlp_hidden=cfg.mlp_hidden,
+                 softmax_scale=0.0)
+    f.update(kw)
+    f.setdefault("mlp_hidden", 256)
+    f.setdefault("softmax_scale", 0.0)
+    return Config(**f)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _want(t: torch.Tensor, name: str, dtype, shape) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _dims(c: Config):
+    N = c.n_hosts * c.block_len
+    return N, c.n_q_heads, c.n_kv_heads, c.head_dim
+
+
+def workspace_bytes(c: Config) -> int:
+    return int(_lib.apb_workspace_bytes(ctypes.byref(c)))
+
+
+def new_workspace(c: Config, device="cuda") -> torch.Tensor:
+    """Zero-filled device workspace of apb_workspace_bytes(c) bytes."""
+    n = workspace_bytes(c)
+    if n == 0:
+        _check(APB_ERR_INVALID_ARG, "apb_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def score_compress(c: Config, q, k, v, w1, b1, w2, b2, scores=None, idx=None, workspace=None,
+                   stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """apb_score_compress: returns (idx [H, Hkv, keep] int32, scores or None)."""
+    N, hq, hkv, d = _dims(c)
+    _want(q, "q", torch.bfloat16, (N, hq, d))
+    _want(k, "k", torch.bfloat16, (N, hkv, d))
+    _want(v, "v", torch.bfloat16, (N, hkv, d))
+    _want(w1, "w1", torch.float32, (hkv, c.mlp_hidden, 3 * d))
+    _want(b1, "b1", torch.float32, (hkv, c.mlp_hidden))
+    _want(w2, "w2", torch.float32, (hkv, c.mlp_hidden))
+    _want(b2, "b2", torch.float32, (hkv,))
+    if scores is not None:
+        _want(scores, "scores", torch.float32, (hkv, N))
+    if idx is None:
+        idx = torch.empty((c.n_hosts, hkv, c.keep), dtype=torch.int32, device=q.device)
+    _want(idx, "idx", torch.int32, (c.n_hosts, hkv, c.keep))
+    if workspace is None:
+        workspace = new_workspace(c, q.device)
+    st = _lib.apb_score_compress(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1),
+                                 _ptr(w2), _ptr(b2), _ptr(scores),
+                                 _ptr(idx) if idx.numel() else None, _ptr(workspace),
+                                 workspace.numel(), _stream(stream))
+    _check(st, "apb_score_compress")
+    return idx, scores
+
+
+def build_passing(c: Config, k, v, idx, pass_k=None, pass_v=None, stream=None):
+    """apb_build_passing: returns (pass_k, pass_v) [Hkv, H*keep, d] bf16."""
+    N, hq, hkv, d = _dims(c)
+    _want(k, "k", torch.bfloat16, (N, hkv, d))
+    _want(v, "v", torch.bfloat16, (N, hkv, d))
+    _want(idx, "idx", torch.int32, (c.n_hosts, hkv, c.keep))
+    shape = (hkv, c.n_hosts * c.keep, d)
+    if pass_k is None:
+        pass_k = torch.empty(shape, dtype=torch.bfloat16, device=k.device)
+    if pass_v is None:
+        pass_v = torch.empty(shape, dtype=torch.bfloat16, device=k.device)
+    _want(pass_k, "pass_k", torch.bfloat16, shape)
+    _want(pass_v, "pass_v", torch.bfloat16, shape)
+    if c.keep == 0:
+        return pass_k, pass_v
+    st = _lib.apb_build_passing(ctypes.byref(c), _ptr(k), _ptr(v), _ptr(idx), _ptr(pass_k),
+                                _ptr(pass_v), _stream(stream))
+    _check(st, "apb_build_passing")
+    return pass_k, pass_v
+
+
+def block_attention(c: Config, q, k, v, pass_k, pass_v, out=None, lse=None, want_lse=False,
+                    workspace=None, stream=None):
+    """apb_block_attention: returns (out [N, Hq, d] bf16, lse [Hq, N] fp32 or None)."""
+    N, hq, hkv, d = _dims(c)
+    _want(q, "q", torch.bfloat16, (N, hq, d))
+    _want(k, "k", torch.bfloat16, (N, hkv, d))
+    _want(v, "v", torch.bfloat16, (N, hkv, d))
+    use_pass = c.keep > 0 and c.n_hosts > 1
+    if use_pass:
+        shape = (hkv, c.n_hosts * c.keep, d)
+        _want(pass_k, "pass_k", torch.bfloat16, shape)
+        _want(pass_v, "pass_v", torch.bfloat16, shape)
+    if out is None:
+        out = torch.empty((N, hq, d), dtype=torch.bfloat16, device=q.device)
+    _want(out, "out", torch.bfloat16, (N, hq, d))
+    if lse is None and want_lse:
+        lse = torch.empty((hq, N), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (hq, N))
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    st = _lib.apb_block_attention(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(pass_k) if use_pass else None,
+                                  _ptr(pass_v) if use_pass else None, _ptr(out), _ptr(lse),
+                                  _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "apb_block_attention")
+    return out, lse
+
+
+def device_status(workspace, stream=None, clear=False) -> int:
+    """apb_device_status: synchronises the stream, returns the status code."""
+    return int(_lib.apb_device_status(_ptr(workspace), _stream(stream), 1 if clear else 0))
+
+
+class Prefill:
+    """One APB prefill over preallocated device buffers: score + compress,
+    build the passing block, block attention.  Buffers are allocated once (by
+    torch) and reused by every call."""
+
+    def __init__(self, c: Config, device="cuda"):
+        N, hq, hkv, d = _dims(c)
+        self.c = c
+        self.workspace = new_workspace(c, device)
+        self.idx = torch.empty((c.n_hosts, hkv, c.keep), dtype=torch.int32, device=device)
+        shape = (hkv, c.n_hosts * c.keep, d)
+        self.pass_k = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.pass_v = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.out = torch.empty((N, hq, d), dtype=torch.bfloat16, device=device)
+
+    def __call__(self, q, k, v, w1, b1, w2, b2, stream=None):
+        score_compress(self.c, q, k, v, w1, b1, w2, b2, idx=self.idx, workspace=self.workspace,
+                       stream=stream)
+        build_passing(self.c, k, v, self.idx, self.pass_k, self.pass_v, stream=stream)
+        block_attention(self.c, q, k, v, self.pass_k, self.pass_v, out=self.out,
+                        workspace=self.workspace, stream=stream)
+        return self.out

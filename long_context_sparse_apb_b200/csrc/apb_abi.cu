@@ -1,0 +1,184 @@
+// C-ABI layer: argument checks, workspace layout, status reporting.
+// Every entry point validates on the host before launching anything and
+// returns an apb_status; no exception or abort crosses the boundary.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "apb_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+apb_status fail(apb_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks the shape rules of apb_config; fills `s` on success.
+apb_status check_config(const apb_config* c, apb::Shape* s) {
+  if (!c) return fail(APB_ERR_INVALID_ARG, "config is NULL");
+  if (c->n_hosts < 1) return fail(APB_ERR_INVALID_ARG, "n_hosts=%d < 1", c->n_hosts);
+  if (c->block_len < 1) return fail(APB_ERR_INVALID_ARG, "block_len=%d < 1", c->block_len);
+  if (c->query_len < 0 || c->query_len > c->anchor_len || c->anchor_len > c->block_len)
+    return fail(APB_ERR_INVALID_ARG, "need 0 <= query_len(%d) <= anchor_len(%d) <= block_len(%d)",
+                c->query_len, c->anchor_len, c->block_len);
+  if (c->keep < 0 || c->keep > c->block_len)
+    return fail(APB_ERR_INVALID_ARG, "need 0 <= keep(%d) <= block_len(%d)", c->keep, c->block_len);
+  if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads != 0)
+    return fail(APB_ERR_INVALID_ARG, "n_q_heads(%d) must be a positive multiple of n_kv_heads(%d)",
+                c->n_q_heads, c->n_kv_heads);
+  if (!(c->softmax_scale == c->softmax_scale))
+    return fail(APB_ERR_INVALID_ARG, "softmax_scale is NaN");
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return fail(APB_ERR_UNSUPPORTED, "head_dim=%d (supported: 64, 128)", c->head_dim);
+  if (c->mlp_hidden != 256)
+    return fail(APB_ERR_UNSUPPORTED, "mlp_hidden=%d (supported: 256)", c->mlp_hidden);
+  long long N = (long long)c->n_hosts * c->block_len;
+  if (N > (1ll << 31) - 1) return fail(APB_ERR_UNSUPPORTED, "sequence length %lld >= 2^31", N);
+  if ((long long)c->n_hosts * c->keep > (1ll << 31) - 1)
+    return fail(APB_ERR_UNSUPPORTED, "n_hosts*keep >= 2^31");
+  s->H = c->n_hosts;
+  s->n = c->block_len;
+  s->A = c->anchor_len;
+  s->keep = c->keep;
+  s->Hq = c->n_q_heads;
+  s->Hkv = c->n_kv_heads;
+  s->d = c->head_dim;
+  s->hidden = c->mlp_hidden;
+  s->N = N;
+  s->scale = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / std::sqrt((float)c->head_dim);
+  return APB_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+apb_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(APB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t apb_workspace_bytes(const apb_config* cfg) {
+  apb::Shape s;
+  if (check_config(cfg, &s) != APB_OK) return 0;
+  return apb::kStatusBytes + round256((size_t)s.Hkv * (size_t)s.N * sizeof(float));
+}
+
+apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* k,
+                              const void* v, const float* w1, const float* b1,
+                              const float* w2, const float* b2, float* scores,
+                              int32_t* idx, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  apb::Shape s;
+  apb_status st = check_config(cfg, &s);
+  if (st != APB_OK) return st;
+  if (!q || !k || !v || !w1 || !b1 || !w2 || !b2 || !workspace)
+    return fail(APB_ERR_INVALID_ARG, "apb_score_compress: NULL input or workspace");
+  if (s.keep > 0 && !idx) return fail(APB_ERR_INVALID_ARG, "apb_score_compress: idx is NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w1) || !aligned16(workspace) ||
+      (scores && !aligned16(scores)) || (idx && !aligned16(idx)))
+    return fail(APB_ERR_INVALID_ARG, "apb_score_compress: pointers must be 16-byte aligned");
+  size_t need = scores ? apb::kStatusBytes : apb_workspace_bytes(cfg);
+  if (ws_bytes < need)
+    return fail(APB_ERR_INVALID_ARG, "apb_score_compress: workspace %zu < %zu bytes", ws_bytes, need);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  float* sc = scores ? scores
+                     : reinterpret_cast<float*>(static_cast<char*>(workspace) + apb::kStatusBytes);
+  cudaError_t e = apb::launch_score(s, q, k, v, w1, b1, w2, b2, sc, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "score kernel");
+  if (s.keep > 0) {
+    e = apb::launch_topk(s, sc, idx, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k kernel");
+  }
+  return APB_OK;
+}
+
+apb_status apb_build_passing(const apb_config* cfg, const void* k, const void* v,
+                             const int32_t* idx, void* pass_k, void* pass_v, void* stream) {
+  apb::Shape s;
+  apb_status st = check_config(cfg, &s);
+  if (st != APB_OK) return st;
+  if (s.keep == 0) return APB_OK;
+  if (!k || !v || !idx || !pass_k || !pass_v)
+    return fail(APB_ERR_INVALID_ARG, "apb_build_passing: NULL pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(pass_k) || !aligned16(pass_v) || !aligned16(idx))
+    return fail(APB_ERR_INVALID_ARG, "apb_build_passing: pointers must be 16-byte aligned");
+  cudaError_t e = apb::launch_gather(s, k, v, idx, pass_k, pass_v,
+                                     reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gather kernel");
+  return APB_OK;
+}
+
+apb_status apb_block_attention(const apb_config* cfg, const void* q, const void* k,
+                               const void* v, const void* pass_k, const void* pass_v,
+                               void* out, float* lse, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  apb::Shape s;
+  apb_status st = check_config(cfg, &s);
+  if (st != APB_OK) return st;
+  if (!q || !k || !v || !out || !workspace)
+    return fail(APB_ERR_INVALID_ARG, "apb_block_attention: NULL q/k/v/out/workspace");
+  bool need_pass = s.keep > 0 && s.H > 1;
+  if (need_pass && (!pass_k || !pass_v))
+    return fail(APB_ERR_INVALID_ARG, "apb_block_attention: NULL pass_k/pass_v with keep > 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace) ||
+      (need_pass && (!aligned16(pass_k) || !aligned16(pass_v))) || (lse && !aligned16(lse)))
+    return fail(APB_ERR_INVALID_ARG, "apb_block_attention: pointers must be 16-byte aligned");
+  if (ws_bytes < apb::kStatusBytes)
+    return fail(APB_ERR_INVALID_ARG, "apb_block_attention: workspace %zu < %zu bytes", ws_bytes,
+                apb::kStatusBytes);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  auto* status = static_cast<apb::DeviceStatus*>(workspace);
+  // clear the in-launch abort flag (the sticky bits stay until cleared)
+  cudaError_t e = cudaMemsetAsync(&status->abort, 0, sizeof(uint32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing abort flag");
+  const char* why = nullptr;
+  e = apb::launch_attention(s, q, k, v, need_pass ? pass_k : nullptr, need_pass ? pass_v : nullptr,
+                            out, lse, status, cs, &why);
+  if (why) return fail(APB_ERR_CUDA, "attention: %s", why);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
+  return APB_OK;
+}
+
+apb_status apb_device_status(void* workspace, void* stream, int clear) {
+  if (!workspace) return fail(APB_ERR_INVALID_ARG, "apb_device_status: NULL workspace");
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  apb::DeviceStatus h{};
+  e = cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading status block");
+  if (clear) {
+    e = cudaMemset(workspace, 0, sizeof(h));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing status block");
+  }
+  if (h.sticky & apb::kErrWaitTimeout)
+    return fail(APB_ERR_TIMEOUT, "a bounded on-chip wait ran out (barrier %u, tile %u)", h.where,
+                h.tile);
+  return APB_OK;
+}
+
+const char* apb_status_string(apb_status status) {
+  switch (status) {
+    case APB_OK: return "APB_OK";
+    case APB_ERR_INVALID_ARG: return "APB_ERR_INVALID_ARG";
+    case APB_ERR_UNSUPPORTED: return "APB_ERR_UNSUPPORTED";
+    case APB_ERR_CUDA: return "APB_ERR_CUDA";
+    case APB_ERR_TIMEOUT: return "APB_ERR_TIMEOUT";
+  }
+  return "APB_ERR_UNKNOWN";
+}
+
+const char* apb_last_error(void) { return g_last_error; }
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// Internal launchers shared by the C-ABI layer (apb_abi.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/apb.h"
+
+namespace apb {
+
+// Status block at the start of every workspace.
+struct DeviceStatus {
+  uint32_t sticky;     // OR of error bits since last clear
+  uint32_t abort;      // set inside a launch once one CTA gave up
+  uint32_t where;      // role/barrier id of the first failed wait
+  uint32_t tile;       // tile index of the first failed wait
+};
+constexpr uint32_t kErrWaitTimeout = 1u;
+constexpr size_t kStatusBytes = 256;
+
+struct Shape {
+  int H, n, A, keep, Hq, Hkv, d, hidden;
+  long long N;
+  float scale;
+};
+
+cudaError_t launch_score(const Shape& s, const void* q, const void* k, const void* v,
+                         const float* w1, const float* b1, const float* w2,
+                         const float* b2, float* scores, cudaStream_t st);
+cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* idx, cudaStream_t st);
+cudaError_t launch_gather(const Shape& s, const void* k, const void* v, const int32_t* idx,
+                          void* pass_k, void* pass_v, cudaStream_t st);
+// Returns cudaSuccess or an error; sets *encode_failed when a TMA descriptor
+// could not be built (reported as APB_ERR_CUDA with a message).
+cudaError_t launch_attention(const Shape& s, const void* q, const void* k, const void* v,
+                             const void* pass_k, const void* pass_v, void* out, float* lse,
+                             DeviceStatus* status, cudaStream_t st, const char** why);
+
+}  // namespace apb

@@ -1,0 +1,131 @@
+"""CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+* scores: fp32 GPU vs fp64 oracle within SCORE_ABS;
+* top-k: identical sets except swaps within a 1e-5 relative score gap of the
+  keep-th largest oracle score; ascending, in range, deterministic;
+* passing block: bit-exact against the oracle's gather of the GPU's indices;
+* attention: max-abs <= 2e-2 and mean-abs <= 2e-3 against the oracle run on
+  the GPU's own index set (so a legal tie swap is not penalised).
+
+Small shapes are compared element by element on every row; the full-size
+workloads run in the launch configuration of bench.py and are compared on
+seeded row samples (edge rows always included).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_sparse_apb_b200 import inputs
+
+from _parity import (check_topk, compare_attention, f32np, oracle_scores, SCORE_ABS)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def apb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_sparse_apb_b200 import _lib
+    return _lib
+
+
+def _to_dev(x):
+    return {k: (v.cuda() if k != "needles" else v) for k, v in x.items()}
+
+
+def _run_gpu(apb, cfg, xd):
+    c = apb.make_config(cfg)
+    N = cfg.seq_len
+    scores = torch.empty((cfg.n_kv_heads, N), dtype=torch.float32, device="cuda")
+    ws = apb.new_workspace(c)
+    idx, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"],
+                                xd["b2"], scores=scores, workspace=ws)
+    pk, pv = apb.build_passing(c, xd["k"], xd["v"], idx)
+    out, lse = apb.block_attention(c, xd["q"], xd["k"], xd["v"], pk, pv, want_lse=True,
+                                   workspace=ws)
+    torch.cuda.synchronize()
+    assert apb.device_status(ws) == apb.APB_OK
+    return scores, idx, pk, pv, out, lse
+
+
+def _check_passing_exact(x, idx_np, pk, pv):
+    k16 = x["k"].view(torch.int16).numpy()
+    v16 = x["v"].view(torch.int16).numpy()
+    rk, rv = oracle.passing_blocks(k16, v16, idx_np.astype(np.int64))
+    assert np.array_equal(pk.view(torch.int16).cpu().numpy(), rk)
+    assert np.array_equal(pv.view(torch.int16).cpu().numpy(), rv)
+
+
+def _full_parity(apb, cfg, x=None):
+    x = inputs.generate(cfg) if x is None else x
+    xd = _to_dev(x)
+    scores, idx, pk, pv, out, lse = _run_gpu(apb, cfg, xd)
+    s_ref = oracle_scores(cfg, x)
+    assert np.abs(scores.cpu().numpy() - s_ref).max() <= SCORE_ABS
+    idx_np = idx.cpu().numpy()
+    if cfg.keep > 0:
+        check_topk(idx_np, s_ref, cfg)
+    _check_passing_exact(x, idx_np, pk, pv)
+    k, v = f32np(x["k"]), f32np(x["v"])
+    pkn, pvn = f32np(pk.cpu()), f32np(pv.cpu())
+    n = cfg.block_len
+    o_all = out.float().cpu().numpy()
+    lse_all = lse.cpu().numpy()
+    for h in range(cfg.n_hosts):
+        rows = np.arange(n)
+        o_ref, lse_ref, _ = oracle.host_attention(f32np(x["q"][h * n:(h + 1) * n]), rows, h, k, v,
+                                                  pkn, pvn, n, cfg.anchor_len, cfg.keep)
+        compare_attention(o_all[h * n:(h + 1) * n], o_ref, f"{cfg.name} host {h}")
+        assert np.abs(lse_all[:, h * n:(h + 1) * n].T - lse_ref).max() < 1e-3
+    return out
+
+
+def test_tiny_workload_every_row(apb):
+    _full_parity(apb, inputs.TINY)
+
+
+SMALL = [
+    # H, n, A, q_len, keep, Hq, Hkv, d
+    (1, 300, 64, 16, 32, 4, 2, 128),     # single host: dense causal
+    (2, 128, 128, 8, 128, 2, 1, 64),     # full anchor, keep all
+    (3, 100, 0, 0, 1, 4, 4, 128),        # no anchor, keep 1, n < one tile
+    (5, 513, 200, 32, 0, 8, 2, 128),     # keep 0, ragged n and anchor
+    (3, 257, 33, 33, 257, 10, 2, 64),    # keep = n, G = 5
+    (4, 384, 96, 16, 130, 4, 1, 128),    # passing tail of 2 rows per 128-tile
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+def test_small_shapes_every_row(apb, shape):
+    H, n, A, ql, keep, hq, hkv, d = shape
+    cfg = inputs.APBConfig("small", n_hosts=H, block_len=n, anchor_len=A, query_len=ql, keep=keep,
+                           n_q_heads=hq, n_kv_heads=hkv, head_dim=d, seed=7 + H * n,
+                           rope_theta=1e4, needles_per_host=2)
+    _full_parity(apb, cfg)
+
+
+def test_deterministic_repeat(apb):
+    cfg = inputs.TINY.replace(n_hosts=3, block_len=640, anchor_len=160, keep=100)
+    xd = _to_dev(inputs.generate(cfg))
+    a = _run_gpu(apb, cfg, xd)
+    b = _run_gpu(apb, cfg, xd)
+    for ta, tb in zip(a, b):
+        assert torch.equal(ta, tb)
+
+
+def test_dense_causal_reduction_on_gpu(apb):
+    # H = 1: the kernel must equal dense causal attention (library, fp32)
+    cfg = inputs.APBConfig("dense", n_hosts=1, block_len=1000, anchor_len=0, query_len=0, keep=0,
+                           n_q_heads=8, n_kv_heads=2, head_dim=128, seed=3)
+    x = inputs.generate(cfg)
+    xd = _to_dev(x)
+    c = apb.make_config(cfg)
+    out, _ = apb.block_attention(c, xd["q"], xd["k"], xd["v"], None, None)
+    q = xd["q"].float().permute(1, 0, 2)[None]
+    k = xd["k"].float().repeat_interleave(4, dim=1).permute(1, 0, 2)[None]
+    v = xd["v"].float().repeat_interleave(4, dim=1).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)[0]
+    err = (out.float().permute(1, 0, 2) - ref).abs()
+    assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3
