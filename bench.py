@@ -1,0 +1,418 @@
+"""Throughput of the APB per-host prefill path on B200.
+
+One step = one whole prefill of one sequence: retaining-head scoring and top-k
+compression (apb_score_compress), the passing block (apb_build_passing) and
+block attention (apb_block_attention), with Q/K/V already resident in HBM.
+Default workload: Llama-3.1-8B attention shapes at 128K (32 q / 8 kv heads,
+d = 128, 8 virtual hosts x 16384 tokens, anchor 2048, keep 2048).
+
+  python bench.py [--gpus N --steps K --warmup W --workload NAME]
+  python bench.py --impl reference ...     # the CPU oracle, bounded sample
+
+N > 1 (one process per GPU under torch.distributed.run): every rank prefills
+its own independent sequence (weak scaling, no collective on the data path);
+the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_sparse_apb_b200 import inputs  # noqa: E402
+
+METRIC = "APB prefill tokens/s at 128K (Llama-8B attn shapes); % bf16 peak; % HBM BW"
+UNIT = "tokens/s"
+
+
+def visible_pairs(cfg) -> int:
+    """(query, key) pairs one q head attends: per host n(n+1)/2 causal, n*A
+    anchor (hosts >= 1), n*h*keep passing."""
+    n, A, keep = cfg.block_len, cfg.anchor_len, cfg.keep
+    return sum(n * (n + 1) // 2 + (n * A if h else 0) + n * h * keep for h in range(cfg.n_hosts))
+
+
+def visited_tile_pairs(cfg) -> int:
+    """Pairs the kernel computes: whole 128x128 tiles (mask applied inside)."""
+    n, A, keep, T = cfg.block_len, cfg.anchor_len, cfg.keep, 128
+    nq = -(-n // T)
+    tot = 0
+    for h in range(cfg.n_hosts):
+        na = -(-A // T) if (h and A) else 0
+        np_ = -(-(h * keep) // T)
+        for t in range(nq):
+            tot += (na + np_ + t + 1) * T * T
+    return tot
+
+
+def attention_flops(cfg, pairs) -> float:
+    return 4.0 * cfg.head_dim * cfg.n_q_heads * pairs
+
+
+def hbm_bytes_compress(cfg) -> int:
+    """Algorithmic bytes of score + top-k + gather (bytes each must move once)."""
+    N, d, hq, hkv = cfg.seq_len, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads
+    H, keep = cfg.n_hosts, cfg.keep
+    return (N * hq * d * 2 + 2 * N * hkv * d * 2 + 2 * N * hkv * 4 + H * hkv * keep * 4
+            + 2 * (2 * H * hkv * keep * d * 2))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[4], f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r[2] > 300.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for r in load:
+            for nm, val in zip(names, r[4]):
+                if val.lower().startswith("active"):
+                    seen.add(nm)
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": load[0][1],
+                "power_w_max": max(r[2] for r in load), "samples": len(load),
+                "reasons": sorted(seen)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def config_dict(cfg, world):
+    return {"workload": cfg.name, "seq_len": cfg.seq_len, "n_hosts": cfg.n_hosts,
+            "block_len": cfg.block_len, "anchor_len": cfg.anchor_len, "keep": cfg.keep,
+            "n_q_heads": cfg.n_q_heads, "n_kv_heads": cfg.n_kv_heads,
+            "head_dim": cfg.head_dim,
+            "parallelism": f"{world} independent sequence(s), one per GPU",
+            "l2": "no flush: each step reads 1.6 GB of Q/K/V (> 126 MB L2)"}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(cfg, x, attn_rows_per_host: int):
+    """Times the oracle on a bounded sample of one prefill and extrapolates to
+    the whole prefill.  Sample: scoring and top-k of host 0's block, the
+    passing block of every host, and attention of `attn_rows_per_host` rows
+    per host on all q heads (rows spread over the block)."""
+    import numpy as np
+    import oracle
+
+    f = lambda t: t.float().numpy()
+    n, H = cfg.block_len, cfg.n_hosts
+    w = [x[k].numpy() for k in ("w1", "b1", "w2", "b2")]
+    t0 = time.perf_counter()
+    s0 = oracle.retaining_scores(f(x["q"][:n]), f(x["k"][:n]), f(x["v"][:n]), *w)
+    t1 = time.perf_counter()
+    idx0 = oracle.compress_indices(s0, 1, n, cfg.keep)
+    t2 = time.perf_counter()
+    idx = np.concatenate([idx0 + h * n for h in range(H)], axis=0)   # stand-in positions
+    k, v = f(x["k"]), f(x["v"])
+    pk, pv = oracle.passing_blocks(k, v, idx)
+    t3 = time.perf_counter()
+    rows = np.linspace(0, n - 1, attn_rows_per_host).astype(np.int64)
+    for h in range(H):
+        oracle.host_attention(f(x["q"][h * n + torch.as_tensor(rows)]), rows, h, k, v, pk, pv, n,
+                              cfg.anchor_len, cfg.keep)
+    t4 = time.perf_counter()
+    total = (t1 - t0) * H + (t2 - t1) * H + (t3 - t2) + (t4 - t3) * (n / attn_rows_per_host)
+    measured = t4 - t0
+    return cfg.seq_len / total, measured
+
+
+def cpu_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        nth = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if nth:
+            return int(max(nth))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, cfg):
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    x = inputs.generate(cfg)
+    rows = args.oracle_rows
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, _ = oracle_sample(cfg, x, rows)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    sample = (f"per step: scoring+top-k of host 0 (x{cfg.n_hosts} hosts), passing block of every "
+              f"host, attention of {rows} rows/host on all {cfg.n_q_heads} q heads "
+              f"(x{cfg.block_len // rows}); NumPy float64")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": cfg.seq_len / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(cfg, args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU path
+
+def run_gpu(args, cfg):
+    from long_context_sparse_apb_b200 import _lib as apb
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    rcfg = cfg.replace(seed=cfg.seed + 1000 * rank)     # independent sequence per rank
+    x = inputs.generate(rcfg)
+    xd = {k: v.to(dev) for k, v in x.items() if k != "needles"}
+    c = apb.make_config(rcfg)
+    run = apb.Prefill(c, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    w = (xd["w1"], xd["b1"], xd["w2"], xd["b2"])
+
+    n_ev = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_ev)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, idx=run.idx,
+                           workspace=run.workspace, stream=stream)
+        if e is not None:
+            e[1].record(stream)
+        apb.build_passing(c, xd["k"], xd["v"], run.idx, run.pass_k, run.pass_v, stream=stream)
+        if e is not None:
+            e[2].record(stream)
+        apb.block_attention(c, xd["q"], xd["k"], xd["v"], run.pass_k, run.pass_v, out=run.out,
+                            workspace=run.workspace, stream=stream)
+        if e is not None:
+            e[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if apb.device_status(run.workspace) != apb.APB_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    status = apb.device_status(run.workspace)
+    if status != apb.APB_OK:
+        raise RuntimeError(f"device status {apb.status_string(status)} after timed steps")
+
+    score_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    gather_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    max_ms = max_over_ranks(elapsed_ms, world)
+    ms_per_step = max_ms / args.steps
+    value = world * cfg.seq_len / (max_ms / 1e3 / args.steps)
+
+    # ---- end to end through the public API with pinned host buffers
+    hx = {k: v.pin_memory() for k, v in x.items() if k != "needles"}
+    hout = torch.empty(run.out.shape, dtype=run.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        for k2 in hx:
+            xd[k2].copy_(hx[k2], non_blocking=True)
+        run(xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"], xd["b2"], stream=stream)
+        hout.copy_(run.out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    e2e_steps = max(2, args.steps // 2)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    barrier(world)
+    e2e_value = world * cfg.seq_len / (e2e_ms / 1e3 / e2e_steps)
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    peaks = load_peaks()
+    pairs = visible_pairs(cfg)
+    tiles = visited_tile_pairs(cfg)
+    fl_alg = attention_flops(cfg, pairs)
+    fl_vis = attention_flops(cfg, tiles)
+    ach = fl_alg / (attn_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    hbm = hbm_bytes_compress(cfg)
+    hbm_ach = hbm / ((score_ms + gather_ms) / 1e3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, meas = oracle_sample(cfg, x, args.oracle_rows)
+        cpu = {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+               "sample": (f"scoring+top-k of host 0 extrapolated x{cfg.n_hosts}, passing block of "
+                          f"all hosts, attention of {args.oracle_rows} rows/host on all heads "
+                          f"extrapolated x{cfg.block_len // args.oracle_rows}; NumPy float64; "
+                          f"{meas:.1f} s measured")}
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if os.path.exists(tpath):
+        tj = json.load(open(tpath))
+        if tj.get("workload") == cfg.name and tj.get("kernel_rev") == apb_kernel_rev():
+            traffic = tj.get("bytes_per_launch")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(cfg, world),
+        "stages_ms": {"score_topk": score_ms, "passing": gather_ms, "attention": attn_ms},
+        "attention": {"tflops_algorithmic": ach, "tflops_visited_tiles": fl_vis / (attn_ms / 1e3) / 1e12,
+                      "frac_visited_of_peak": fl_vis / (attn_ms / 1e3) / 1e12 / peak},
+        "compress_stages": {"bytes": hbm, "gbs": hbm_ach, "frac_of_hbm_peak": hbm_ach / peaks["hbm_gbs"]},
+        "roofline": {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                     "frac": ach / peak, "traffic": traffic,
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel runs "
+                                    f"{attn_ms:.1f} ms per launch, back to back)"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * (4 if cfg.keep > 0 else 2),
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def apb_kernel_rev() -> str:
+    """Hash of the attention kernel source: ncu traffic counters only apply to
+    the revision they were taken on."""
+    import hashlib
+    p = os.path.join(ROOT, "long_context_sparse_apb_b200", "csrc", "attention.cu")
+    return hashlib.sha1(open(p, "rb").read()).hexdigest()[:12]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="llama8b_128k", choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--oracle-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = inputs.CONFIGS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_gpu(args, cfg)
+
+
+if __name__ == "__main__":
+    main()
