@@ -124,6 +124,30 @@ apb_status apb_block_attention(const apb_config* cfg, const void* q, const void*
                                void* out, float* lse, void* workspace, size_t ws_bytes,
                                void* stream);
 
+/* No counterpart in the paper: an allocation-free variant of
+ * apb_score_compress, for callers that cannot hand this library any device
+ * memory besides the tensors themselves (a host framework whose allocator
+ * owns all device memory and only exposes inputs and outputs to plug-ins, or
+ * a service that must not allocate after start-up).  Same computation,
+ * arguments and outputs as apb_score_compress with scores == NULL, but the
+ * fp32 scores live in a fixed device array inside the library instead of a
+ * workspace; nothing is allocated by the call.
+ *   - The array holds apb_score_compress_static_max_floats() floats (16 MiB);
+ *     every GPU that loads the library keeps it until the process exits.
+ *     n_kv_heads * N above that returns APB_ERR_UNSUPPORTED.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Each call writes every score it reads, so nothing needs clearing, but
+ *     two calls whose kernels overlap on the GPU (other streams or threads)
+ *     race on it: serialise them. */
+size_t apb_score_compress_static_max_floats(void);
+apb_status apb_score_compress_static(const apb_config* cfg, const void* q, const void* k,
+                                     const void* v, const float* w1, const float* b1,
+                                     const float* w2, const float* b2, int32_t* idx,
+                                     void* stream);
+
 /* Synchronises `stream`, then reads the status block of `workspace`:
  * APB_ERR_TIMEOUT if a kernel recorded a bounded wait that ran out since the
  * block was last cleared, else APB_OK (APB_ERR_CUDA if the reads fail).

@@ -43,6 +43,10 @@ _lib.apb_build_passing.argtypes = [ctypes.POINTER(Config)] + [_P] * 6
 _lib.apb_build_passing.restype = ctypes.c_int
 _lib.apb_block_attention.argtypes = [ctypes.POINTER(Config)] + [_P] * 8 + [ctypes.c_size_t, _P]
 _lib.apb_block_attention.restype = ctypes.c_int
+_lib.apb_score_compress_static.argtypes = [ctypes.POINTER(Config)] + [_P] * 9
+_lib.apb_score_compress_static.restype = ctypes.c_int
+_lib.apb_score_compress_static_max_floats.argtypes = []
+_lib.apb_score_compress_static_max_floats.restype = ctypes.c_size_t
 _lib.apb_device_status.argtypes = [_P, _P, ctypes.c_int]
 _lib.apb_device_status.restype = ctypes.c_int
 _lib.apb_status_string.argtypes = [ctypes.c_int]
@@ -150,6 +154,27 @@ def score_compress(c: Config, q, k, v, w1, b1, w2, b2, scores=None, idx=None, wo
                                  workspace.numel(), _stream(stream))
     _check(st, "apb_score_compress")
     return idx, scores
+
+
+def score_compress_static(c: Config, q, k, v, w1, b1, w2, b2, idx=None, stream=None):
+    """apb_score_compress_static: the allocation-free variant (scores kept in
+    the library's fixed device array); returns idx [H, Hkv, keep] int32."""
+    N, hq, hkv, d = _dims(c)
+    _want(q, "q", torch.bfloat16, (N, hq, d))
+    _want(k, "k", torch.bfloat16, (N, hkv, d))
+    _want(v, "v", torch.bfloat16, (N, hkv, d))
+    _want(w1, "w1", torch.float32, (hkv, c.mlp_hidden, 3 * d))
+    _want(b1, "b1", torch.float32, (hkv, c.mlp_hidden))
+    _want(w2, "w2", torch.float32, (hkv, c.mlp_hidden))
+    _want(b2, "b2", torch.float32, (hkv,))
+    if idx is None:
+        idx = torch.empty((c.n_hosts, hkv, c.keep), dtype=torch.int32, device=q.device)
+    _want(idx, "idx", torch.int32, (c.n_hosts, hkv, c.keep))
+    st = _lib.apb_score_compress_static(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(w1),
+                                        _ptr(b1), _ptr(w2), _ptr(b2),
+                                        _ptr(idx) if idx.numel() else None, _stream(stream))
+    _check(st, "apb_score_compress_static")
+    return idx
 
 
 def build_passing(c: Config, k, v, idx, pass_k=None, pass_v=None, stream=None):
