@@ -2,27 +2,35 @@
 // computation over the anchor block, the passing block and the local block;
 // the passing block is not kept afterwards).
 //
-// One CTA computes one 128-row query tile of one q head of one host.  Its KV
-// sequence is three ranges, walked as 128-row tiles:
+// One CTA computes two consecutive 128-row query tiles (A, B) of one q head
+// of one host.  Their KV sequence is three ranges walked as 128-row tiles:
 //   anchor  : k[0:A, g]             (hosts h >= 1)      full visibility
 //   passing : pass_k[g, 0:h*keep]                       full visibility
-//   local   : k[h*n : h*n + q0 + 128, g]                causal, diagonal kept
-// so masked tiles beyond the diagonal are never visited and only the last
-// tile of each range needs a mask.
+//   local   : k[h*n : h*n + qB0 + 128, g]               causal, diagonal kept
+// Tile A stops one KV tile earlier than tile B (its own diagonal); tiles
+// beyond a diagonal are never visited and only the last tile of each range
+// needs a mask.  Every K and V tile in shared memory feeds both query tiles.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax + epilogue; thread r owns query row r, which is also
-//              TMEM lane r of every accumulator;
-//   warp 4     TMA producer (Q once, then K and V tiles into 2-stage rings);
-//   warp 5     TMEM allocator and the single UMMA-issuing thread.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+d).
-// Per KV tile j:   S(j) = Q K(j)^T            (tcgen05.mma, into S[j&1])
-//                  softmax reads S(j), writes P(j) (bf16, SW128 K-major) to
-//                  shared memory, rescales O in TMEM when the running max
-//                  grew by more than 2^8 (lazy rescaling), signals P_FULL;
-//                  O += P(j) V(j)          (A = P from smem, B = V MN-major)
-// The MMA thread issues S(j+2) right after PV(j), so the tensor core works
-// on the next score tile while the softmax warps process the current one.
+// Warp roles (320 threads):
+//   warps 0-3  softmax + epilogue of query tile A (thread r owns row r, which
+//              is TMEM lane r of S_A, P_A and O_A);
+//   warps 4-7  the same for query tile B;
+//   warp 8     TMA producer (Q_A, Q_B once, K and V tiles into 2-stage rings);
+//   warp 9     TMEM allocator and the single UMMA-issuing thread.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// P_A (bf16, two per 32-bit column) overwrites S_A columns [0,64) once the
+// softmax has read S_A; likewise P_B in S_B.
+// Per KV tile j and query tile i:
+//   S_i(j) = Q_i K(j)^T         tcgen05.mma, A and B from shared memory
+//   softmax_i reads S_i(j), rescales O_i in TMEM when the running max grew by
+//   more than 2^8 (lazy rescaling), writes P_i(j) to TMEM, signals P_FULL_i
+//   O_i += P_i(j) V(j)          tcgen05.mma, A = P_i from TMEM, B = V
+// The MMA thread issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while one
+// softmax warpgroup works on its tile the tensor core serves the other.
+// tcgen05 MMAs of one thread execute in issue order, so S_i(j+1) overwrites
+// P_i(j) only after PV_i(j) has read it, and the commit that signals
+// S_i(j+1) also covers PV_i(j): when the softmax sees S_i(j+1), O_i is
+// stable and may be rescaled.
 //
 // Every mbarrier wait is bounded (wall-clock limit plus a launch-wide abort
 // flag); a wait that runs out records an error in the status block, the CTA
@@ -39,7 +47,7 @@ namespace apb {
 namespace {
 
 constexpr int kRows = 128;                    // query rows per tile = KV rows per tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
@@ -50,22 +58,20 @@ enum Bar {
   K_EMPTY = 3,   // 2
   V_FULL = 5,    // 2
   V_EMPTY = 7,   // 2
-  S_FULL = 9,    // 2
-  P_FULL = 11,
-  O_DONE = 12,
-  DRAIN = 13,
-  NUM_BARS = 14
+  S_FULL = 9,    // per query tile (A, B)
+  P_FULL = 11,   // per query tile
+  O_FINAL = 13,  // per query tile
+  DRAIN = 15,
+  NUM_BARS = 16
 };
 
 template <int D>
 struct Layout {
   static constexpr int kTile = kRows * D * 2;   // bytes of one Q/K/V tile
-  static constexpr int kP = kRows * kRows * 2;  // bytes of the P tile
-  static constexpr int kQ = 0;
-  static constexpr int kK0 = kTile;
-  static constexpr int kV0 = 3 * kTile;
-  static constexpr int kPoff = 5 * kTile;
-  static constexpr int kBars = kPoff + kP;
+  static constexpr int kQ = 0;                  // Q_A, Q_B
+  static constexpr int kK0 = 2 * kTile;         // K stages
+  static constexpr int kV0 = 4 * kTile;         // V stages
+  static constexpr int kBars = 6 * kTile;
   static constexpr int kBytes = kBars + 256;
 };
 // Both head sizes request the d = 128 footprint so that one CTA runs per SM
@@ -73,7 +79,7 @@ struct Layout {
 constexpr int kSmemBytes = Layout<128>::kBytes + 1024;
 
 struct Params {
-  int H, n, A, keep, Hq, Hkv, G, n_qtiles;
+  int H, n, A, keep, Hq, Hkv, G, n_ctas_per_host;
   long long N;
   float scale_log2;
   __nv_bfloat16* out;
@@ -122,38 +128,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 16);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
   uint32_t* s_flags = s_tmem + 1;   // [0]: launch already aborted, [1]: constant 0
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   // heavy units first: the last query tiles of the last hosts
-  const int t = p.n_qtiles - 1 - (int)blockIdx.x;
+  const int u = p.n_ctas_per_host - 1 - (int)blockIdx.x;
   const int head = (int)blockIdx.y;
   const int h = p.H - 1 - (int)blockIdx.z;
   const int g = head / p.G;
-  const int q0 = t * kRows;
+  const int qA0 = 2 * u * kRows;                 // first local row of tile A
   const int na = (h >= 1 && p.A > 0) ? (p.A + kRows - 1) / kRows : 0;
   const int P = h * p.keep;
   const int np = (P + kRows - 1) / kRows;
-  const int T = na + np + t + 1;
-  const int local_row0 = h * p.n;        // first K row of this host's block
+  const int TA = na + np + 2 * u + 1;            // KV tiles of query tile A
+  const int TB = (qA0 + kRows < p.n) ? TA + 1 : 0;   // of tile B (0: beyond the block)
+  const int Tmax = TB > 0 ? TB : TA;
+  const int local_row0 = h * p.n;                // first K row of this host's block
 
   const volatile uint32_t* gabort = &p.status->abort;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM_BARS; ++i) ptx::mbar_init(&bars[i], 1);
     ptx::mbar_init(&bars[P_FULL], 128);
+    ptx::mbar_init(&bars[P_FULL + 1], 128);
     ptx::fence_mbar_init();
     s_flags[0] = *gabort;
     s_flags[1] = 0u;
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tmem_alloc(s_tmem, 512);
     ptx::tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     ptx::tma_prefetch_desc(&mQ);
     ptx::tma_prefetch_desc(&mK);
     ptx::tma_prefetch_desc(&mV);
@@ -167,21 +176,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const volatile uint32_t* never = s_flags + 1;
   const bool skip = s_flags[0] != 0u;
 
-  uint8_t* sQ = smem + L::kQ;
+  uint8_t* sQ = smem + L::kQ;     // tile i at sQ + i * kTile
   uint8_t* sK0 = smem + L::kK0;   // stage s at sK0 + s * kTile
   uint8_t* sV0 = smem + L::kV0;
-  uint8_t* sP = smem + L::kPoff;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !skip) {
       int lastK[2] = {-1, -1}, lastV[2] = {-1, -1};   // parity of the last load per slot
-      ptx::mbar_arrive_expect_tx(&bars[Q_FULL], L::kTile);
+      ptx::mbar_arrive_expect_tx(&bars[Q_FULL], (TB > 0 ? 2 : 1) * L::kTile);
+      for (int i = 0; i < (TB > 0 ? 2 : 1); ++i) {
 #pragma unroll
-      for (int kb = 0; kb < D / 64; ++kb)
-        ptx::tma_load_3d(sQ + kb * (kRows * 128), &mQ, &bars[Q_FULL], kb * 64, head,
-                         local_row0 + q0);
-      for (int j = 0; j < T; ++j) {
+        for (int kb = 0; kb < D / 64; ++kb)
+          ptx::tma_load_3d(sQ + i * L::kTile + kb * (kRows * 128), &mQ, &bars[Q_FULL], kb * 64,
+                           head, local_row0 + qA0 + i * kRows);
+      }
+      for (int j = 0; j < Tmax; ++j) {
         const int s = j & 1;
         const uint32_t par = (j >> 1) & 1;
         if (!ptx::mbar_wait_bounded(&bars[K_EMPTY + s], par ^ 1, gabort, kWaitLimitNs)) {
@@ -189,14 +199,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         ptx::mbar_arrive_expect_tx(&bars[K_FULL + s], L::kTile);
-        load_kv_tile<D>(&mK, &mPK, sK0 + s * L::kTile, &bars[K_FULL + s], j, na, np, g, local_row0);
+        load_kv_tile<D>(&mK, &mPK, sK0 + s * L::kTile, &bars[K_FULL + s], j, na, np, g,
+                        local_row0);
         lastK[s] = (int)par;
         if (!ptx::mbar_wait_bounded(&bars[V_EMPTY + s], par ^ 1, gabort, kWaitLimitNs)) {
           record_failure(p.status, 42 + s, j);
           break;
         }
         ptx::mbar_arrive_expect_tx(&bars[V_FULL + s], L::kTile);
-        load_kv_tile<D>(&mV, &mPV, sV0 + s * L::kTile, &bars[V_FULL + s], j, na, np, g, local_row0);
+        load_kv_tile<D>(&mV, &mPV, sV0 + s * L::kTile, &bars[V_FULL + s], j, na, np, g,
+                        local_row0);
         lastV[s] = (int)par;
       }
       // drain: every load issued must have landed before the CTA exits
@@ -206,59 +218,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lastV[s] >= 0) ptx::mbar_wait_bounded(&bars[V_FULL + s], lastV[s], never, kWaitLimitNs);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && !skip) {
       const uint32_t idesc_s = ptx::idesc_bf16_f32(kRows, kRows, 0);
       const uint32_t idesc_pv = ptx::idesc_bf16_f32(kRows, D, 1);
-      const uint32_t aQ = ptx::smem_u32(sQ), aP = ptx::smem_u32(sP);
+      const uint32_t aQ = ptx::smem_u32(sQ);
       const uint32_t aK0 = ptx::smem_u32(sK0), aV0 = ptx::smem_u32(sV0);
-      const uint32_t tO = tmem + 256;
-      bool ok = ptx::mbar_wait_bounded(&bars[Q_FULL], 0, gabort, kWaitLimitNs);
-      if (!ok) record_failure(p.status, 50, 0);
+      const int T[2] = {TA, TB};
 
-      auto issue_s = [&](int jj) -> bool {
+      // S_i(jj) = Q_i K(jj)^T into S_i; K(jj) must have landed
+      auto issue_s = [&](int i, int jj) {
         const int s = jj & 1;
-        if (!ptx::mbar_wait_bounded(&bars[K_FULL + s], (jj >> 1) & 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 51 + s, jj);
-          return false;
-        }
-        ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
-          ptx::umma_bf16_ss(tmem + 128 * s, ptx::sdesc_sw128(aQ + off, 16, 1024),
+          ptx::umma_bf16_ss(tmem + 128 * i, ptx::sdesc_sw128(aQ + i * L::kTile + off, 16, 1024),
                             ptx::sdesc_sw128(aK0 + s * L::kTile + off, 16, 1024), idesc_s,
                             kk > 0);
         }
-        ptx::umma_commit(&bars[K_EMPTY + s]);
-        ptx::umma_commit(&bars[S_FULL + s]);
+        ptx::umma_commit(&bars[S_FULL + i]);
+      };
+      auto wait_k = [&](int jj) -> bool {
+        if (!ptx::mbar_wait_bounded(&bars[K_FULL + (jj & 1)], (jj >> 1) & 1, gabort,
+                                    kWaitLimitNs)) {
+          record_failure(p.status, 51 + (jj & 1), jj);
+          return false;
+        }
+        ptx::tc_fence_after();
         return true;
       };
 
-      if (ok) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < T; ++j) {
+      bool ok = ptx::mbar_wait_bounded(&bars[Q_FULL], 0, gabort, kWaitLimitNs);
+      if (!ok) record_failure(p.status, 50, 0);
+      if (ok) ok = wait_k(0);
+      if (ok) {
+        issue_s(0, 0);
+        if (TB > 0) issue_s(1, 0);
+        ptx::umma_commit(&bars[K_EMPTY]);
+      }
+      for (int j = 0; ok && j < Tmax; ++j) {
         const int s = j & 1;
-        if (!ptx::mbar_wait_bounded(&bars[P_FULL], j & 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 53, j);
-          break;
-        }
         if (!ptx::mbar_wait_bounded(&bars[V_FULL + s], (j >> 1) & 1, gabort, kWaitLimitNs)) {
           record_failure(p.status, 54 + s, j);
           break;
         }
         ptx::tc_fence_after();
+        bool k_next = false;   // K(j+1) waited for
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (j >= T[i]) continue;
+          if (!ptx::mbar_wait_bounded(&bars[P_FULL + i], j & 1, gabort, kWaitLimitNs)) {
+            record_failure(p.status, 56 + i, j);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t tP = tmem + 128 * i;
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {
-          const uint32_t offp = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
-          ptx::umma_bf16_ss(tO, ptx::sdesc_sw128(aP + offp, 16, 1024),
-                            ptx::sdesc_sw128(aV0 + s * L::kTile + kk * 2048, kRows * 128, 1024), idesc_pv,
-                            (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            ptx::umma_bf16_ts(tmem + 256 + 128 * i, tP + kk * 8,
+                              ptx::sdesc_sw128(aV0 + s * L::kTile + kk * 2048, kRows * 128, 1024),
+                              idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          if (j + 1 < T[i]) {
+            if (!k_next) {
+              if (!(ok = wait_k(j + 1))) break;
+              k_next = true;
+            }
+            issue_s(i, j + 1);
+          } else {
+            ptx::umma_commit(&bars[O_FINAL + i]);
+          }
         }
+        if (!ok) break;
         ptx::umma_commit(&bars[V_EMPTY + s]);
-        ptx::umma_commit(&bars[O_DONE]);
-        if (j + 2 < T) ok = issue_s(j + 2);
+        if (k_next) ptx::umma_commit(&bars[K_EMPTY + ((j + 1) & 1)]);
       }
       // drain every MMA issued so far
       ptx::umma_commit(&bars[DRAIN]);
@@ -266,29 +299,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (!skip) {
     // ------------------------------------------------------------ softmax
-    const int row = threadIdx.x;                       // 0..127
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t tS0 = tmem + lane_off;   // S buffer s at tS0 + 128 * s
-    const uint32_t tO = tmem + 256 + lane_off;
-    uint8_t* prow = sP + row * 128;
-    const int swz = row & 7;
+    const int i = warp >> 2;                           // query tile A (0) or B (1)
+    const int row = threadIdx.x & 127;
+    const int T = i == 0 ? TA : TB;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 128 * i + lane_off;     // S_i, and P_i in its first 64 columns
+    const uint32_t tO = tmem + 256 + 128 * i + lane_off;
+    const int q0 = qA0 + i * kRows;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
-      const int s = j & 1;
-      ok = ptx::mbar_wait_bounded(&bars[S_FULL + s], (j >> 1) & 1, gabort, kWaitLimitNs);
+      ok = ptx::mbar_wait_bounded(&bars[S_FULL + i], j & 1, gabort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) record_failure(p.status, 60 + s, j);
+        if (lane == 0) record_failure(p.status, 60 + i, j);
         ok = false;
         break;
       }
       ptx::tc_fence_after();
       uint32_t sr[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t* r = sr + 32 * c;
-        APB_TMEM_LD32(tS0 + 128 * s + 32 * c, r);
-      }
+      APB_TMEM_LD128(tS, sr);
       // visible columns of this row in this tile
       int lim;
       if (j < na) {
@@ -305,11 +334,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[i]);
+      for (int x = 0; x < 8; ++x) mx[x] = __uint_as_float(sr[x]);
 #pragma unroll
       for (int c = 8; c < kRows; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
-      float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_tile = tmax * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -332,73 +361,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk[c] = ptx::pack_bf16x2(p0, p1);
       }
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
-      // P buffer and O are free once PV(j-1) has completed
-      if (j > 0) {
-        ok = ptx::mbar_wait_bounded(&bars[O_DONE], (j - 1) & 1, gabort, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, ok)) {
-          if (lane == 0) record_failure(p.status, 62, j);
-          ok = false;
-          break;
-        }
-      }
+      // O_i is stable here: the commit that signalled S_i(j) covers PV_i(j-1)
       if (__any_sync(0xffffffffu, rescale)) {
-        ptx::tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           APB_TMEM_LD32(tO + 32 * c, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
           APB_TMEM_ST32(tO + 32 * c, o);
         }
-        ptx::tmem_st_wait();
       }
-#pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        const int kb = c8 >> 3, ch = c8 & 7;
-        uint4 val = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
-        *reinterpret_cast<uint4*>(prow + kb * (kRows * 128) + ((ch ^ swz) << 4)) = val;
-      }
-      ptx::fence_proxy_async_smem();
+      APB_TMEM_ST64(tS, pk);
+      ptx::tmem_st_wait();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars[P_FULL]);
+      ptx::mbar_arrive(&bars[P_FULL + i]);
     }
-    if (ok) {
-      ok = ptx::mbar_wait_bounded(&bars[O_DONE], (T - 1) & 1, gabort, kWaitLimitNs);
+    if (ok && T > 0) {
+      ok = ptx::mbar_wait_bounded(&bars[O_FINAL + i], 0, gabort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) record_failure(p.status, 63, T);
+        if (lane == 0) record_failure(p.status, 63 + i, T);
         ok = false;
       }
-    }
-    if (ok) {
-      ptx::tc_fence_after();
-      const float inv = 1.0f / l;
-      const bool valid = q0 + row < p.n;
-      const long long tok = (long long)local_row0 + q0 + row;
-      __nv_bfloat16* orow = p.out + (tok * p.Hq + head) * D;
+      if (ok) {
+        ptx::tc_fence_after();
+        const float inv = 1.0f / l;
+        const bool valid = q0 + row < p.n;
+        const long long tok = (long long)local_row0 + q0 + row;
+        __nv_bfloat16* orow = p.out + (tok * p.Hq + head) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        APB_TMEM_LD32(tO + 32 * c, o);
-        uint32_t w[16];
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          APB_TMEM_LD32(tO + 32 * c, o);
+          uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = ptx::pack_bf16x2(__uint_as_float(o[2 * i]) * inv,
-                                  __uint_as_float(o[2 * i + 1]) * inv);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+          for (int x = 0; x < 16; ++x)
+            w[x] = ptx::pack_bf16x2(__uint_as_float(o[2 * x]) * inv,
+                                    __uint_as_float(o[2 * x + 1]) * inv);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            for (int x = 0; x < 4; ++x)
+              dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+          }
         }
+        if (p.lse && valid)
+          p.lse[(long long)head * p.N + tok] = (m + __log2f(l)) * 0.6931471805599453f;
       }
-      if (p.lse && valid) p.lse[(long long)head * p.N + tok] = (m + __log2f(l)) * 0.6931471805599453f;
     }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
   }
@@ -469,7 +484,7 @@ cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v
   p.Hq = s.Hq;
   p.Hkv = s.Hkv;
   p.G = s.Hq / s.Hkv;
-  p.n_qtiles = (s.n + kRows - 1) / kRows;
+  p.n_ctas_per_host = ((s.n + kRows - 1) / kRows + 1) / 2;
   p.N = s.N;
   p.scale_log2 = s.scale * kLog2e;
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -478,7 +493,7 @@ cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v
   cudaError_t e = cudaFuncSetAttribute(apb_attention_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_qtiles, s.Hq, s.H);
+  dim3 grid(p.n_ctas_per_host, s.Hq, s.H);
   apb_attention_kernel<D><<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, mPK, mPV, p);
   return cudaGetLastError();
 }
