@@ -380,7 +380,7 @@ def run_gpu(args, cfg):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * (4 if cfg.keep > 0 else 2),
+        "gpu_launches": args.steps * (5 if cfg.keep > 0 else 3),
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)

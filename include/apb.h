@@ -76,10 +76,11 @@ typedef struct apb_config {
 } apb_config;
 
 /* Bytes of device workspace that apb_score_compress and apb_block_attention
- * need: a 256-byte status block, plus Hkv*N*4 bytes (rounded up to 256) for
- * the scores when apb_score_compress is given scores == NULL.  Returns 0 for
- * a NULL or invalid config.  The caller zero-fills a workspace once before
- * its first use (the status block must start at zero). */
+ * need: a 256-byte status block, then the bf16 hi/lo split of W1
+ * (Hkv*hidden*3d*4 bytes, rounded up to 256), then Hkv*N*4 bytes (rounded up
+ * to 256) for the scores when apb_score_compress is given scores == NULL.
+ * Returns 0 for a NULL or invalid config.  The caller zero-fills a workspace
+ * once before its first use (the status block must start at zero). */
 size_t apb_workspace_bytes(const apb_config* cfg);
 
 /* Step 1 (main features: KV compression with retaining heads; technical
@@ -92,7 +93,12 @@ size_t apb_workspace_bytes(const apb_config* cfg);
  *   w1 [Hkv, hidden, 3d], b1 [Hkv, hidden], w2 [Hkv, hidden], b2 [Hkv]: fp32
  *   scores [Hkv, N] fp32 (out, may be NULL: then held in the workspace)
  *   idx [H, Hkv, keep] int32 (out): global positions, ascending per (h, g)
- *   workspace/ws_bytes: at least apb_workspace_bytes(cfg) bytes. */
+ *   workspace/ws_bytes: apb_workspace_bytes(cfg) bytes, or, when scores is
+ *   given, the status block and the weight split only.
+ * The products run on the tensor cores in bf16 with fp32 accumulation on an
+ * exact rewrite: each fp32 weight is split into bf16 hi + lo, and the group
+ * mean is folded into the q weights (W1_q / G applied to every q head), so
+ * the only rounding beyond fp32 is the 2^-17 relative residual of the split. */
 apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* k,
                               const void* v, const float* w1, const float* b1,
                               const float* w2, const float* b2, float* scores,
@@ -130,15 +136,18 @@ apb_status apb_block_attention(const apb_config* cfg, const void* q, const void*
  * owns all device memory and only exposes inputs and outputs to plug-ins, or
  * a service that must not allocate after start-up).  Same computation,
  * arguments and outputs as apb_score_compress with scores == NULL, but the
- * fp32 scores live in a fixed device array inside the library instead of a
- * workspace; nothing is allocated by the call.
- *   - The array holds apb_score_compress_static_max_floats() floats (16 MiB);
- *     every GPU that loads the library keeps it until the process exits.
- *     n_kv_heads * N above that returns APB_ERR_UNSUPPORTED.
- *   - The first call on each device looks up the array's device address
+ * fp32 scores and the weight split live in fixed device arrays inside the
+ * library instead of a workspace; nothing is allocated by the call.
+ *   - The arrays hold apb_score_compress_static_max_floats() floats (16 MiB)
+ *     of scores and 8 MiB of split weights; every GPU that loads the library
+ *     keeps them until the process exits.  n_kv_heads * N above the first,
+ *     or n_kv_heads * mlp_hidden * 3 * head_dim * 4 bytes above the second,
+ *     returns APB_ERR_UNSUPPORTED.  A bounded wait that runs out inside
+ *     this variant is not reported (its status block is private).
+ *   - The first call on each device looks up the arrays' device addresses
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
- *   - All calls share the one array and it keeps the last call's contents.
+ *   - All calls share the arrays and they keep the last call's contents.
  *     Each call writes every score it reads, so nothing needs clearing, but
  *     two calls whose kernels overlap on the GPU (other streams or threads)
  *     race on it: serialise them. */

@@ -71,7 +71,8 @@ extern "C" {
 size_t apb_workspace_bytes(const apb_config* cfg) {
   apb::Shape s;
   if (check_config(cfg, &s) != APB_OK) return 0;
-  return apb::kStatusBytes + round256((size_t)s.Hkv * (size_t)s.N * sizeof(float));
+  return apb::kStatusBytes + round256(apb::weight_split_bytes(s)) +
+         round256((size_t)s.Hkv * (size_t)s.N * sizeof(float));
 }
 
 apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* k,
@@ -88,13 +89,19 @@ apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w1) || !aligned16(workspace) ||
       (scores && !aligned16(scores)) || (idx && !aligned16(idx)))
     return fail(APB_ERR_INVALID_ARG, "apb_score_compress: pointers must be 16-byte aligned");
-  size_t need = scores ? apb::kStatusBytes : apb_workspace_bytes(cfg);
+  const size_t wsplit = round256(apb::weight_split_bytes(s));
+  const size_t need = scores ? apb::kStatusBytes + wsplit : apb_workspace_bytes(cfg);
   if (ws_bytes < need)
     return fail(APB_ERR_INVALID_ARG, "apb_score_compress: workspace %zu < %zu bytes", ws_bytes, need);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  float* sc = scores ? scores
-                     : reinterpret_cast<float*>(static_cast<char*>(workspace) + apb::kStatusBytes);
-  cudaError_t e = apb::launch_score(s, q, k, v, w1, b1, w2, b2, sc, cs);
+  char* ws = static_cast<char*>(workspace);
+  auto* status = reinterpret_cast<apb::DeviceStatus*>(ws);
+  float* sc = scores ? scores : reinterpret_cast<float*>(ws + apb::kStatusBytes + wsplit);
+  cudaError_t e = cudaMemsetAsync(&status->abort, 0, sizeof(uint32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing abort flag");
+  const char* why = nullptr;
+  e = apb::launch_score(s, q, k, v, w1, b1, w2, b2, sc, ws + apb::kStatusBytes, status, cs, &why);
+  if (why) return fail(APB_ERR_CUDA, "score: %s", why);
   if (e != cudaSuccess) return cuda_fail(e, "score kernel");
   if (s.keep > 0) {
     e = apb::launch_topk(s, sc, idx, cs);

@@ -1,6 +1,7 @@
 // Internal launchers shared by the C-ABI layer (apb_abi.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -24,9 +25,20 @@ struct Shape {
   float scale;
 };
 
+// 3-D bf16 tensor map with 128-byte swizzle, zero fill out of bounds.
+bool encode_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                    uint32_t b2);
+
+// Bytes of the bf16 hi/lo split of W1 kept in the workspace.
+inline size_t weight_split_bytes(const Shape& s) {
+  return (size_t)s.Hkv * 2 * s.hidden * 3 * s.d * 2;
+}
+
 cudaError_t launch_score(const Shape& s, const void* q, const void* k, const void* v,
                          const float* w1, const float* b1, const float* w2,
-                         const float* b2, float* scores, cudaStream_t st);
+                         const float* b2, float* scores, void* wsplit, DeviceStatus* status,
+                         cudaStream_t st, const char** why);
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* idx, cudaStream_t st);
 cudaError_t launch_gather(const Shape& s, const void* k, const void* v, const int32_t* idx,
                           void* pass_k, void* pass_v, cudaStream_t st);

@@ -1,163 +1,269 @@
-// Retaining-head stand-in scores ("APB 的主要功能": each host compresses its
-// KV with retaining heads).  For token t and kv head g:
-//     x = [k[t,g] ; v[t,g] ; mean_{j in group g} q[t,j]]         (3d, fp32)
+// Retaining-head stand-in scores on the tensor cores ("APB 的主要功能": each
+// host compresses its KV with retaining heads).  For token t and kv head g:
+//     x = [k[t,g] ; v[t,g] ; mean_{j in group g} q[t,j]]          (3d)
 //     s[g,t] = w2[g] . SiLU(W1[g] x + b1[g]) + b2[g]
-// computed in fp32 on the CUDA cores (the top-k that follows needs fp32-level
-// ordering of the scores).
 //
-// Tiling: a CTA owns 64 tokens of one kv head and all 256 hidden units, i.e.
-// a [64 x 3d] x [3d x 256] product.  The 3d input features stream through
-// shared memory in chunks of 32: the token chunk is gathered from bf16 K, V
-// and the G q heads of the group (averaged in fp32), the W1 chunk is read
-// along its contiguous feature axis and stored transposed.  Each of the 256
-// threads accumulates a 4-token x 16-hidden register tile; the epilogue
-// applies b1, SiLU and w2 and reduces the 16 hidden groups with shuffles.
+// The product W1 x must be fp32-accurate (the top-k that follows orders the
+// scores), while the tensor cores multiply bf16.  Two exact rewrites make that
+// possible:
+//   * the group mean is folded into the weights: W1_q (1/G) sum_j q_j =
+//     sum_j (W1_q / G) q_j, so every input row is an exact bf16 row of K, V or
+//     one q head, and no averaged (inexact) q ever exists;
+//   * each fp32 weight w is split into bf16 hi + lo (hi = rn(w), lo = rn(w -
+//     hi)), leaving |w - hi - lo| <= 2^-17 |w|; both halves are multiplied
+//     with fp32 accumulation.
+// So Z = X W1^T is computed as sum over the 2 + G input blocks of
+// X_b (Wh_b + Wl_b)^T with UMMA (M = 128 tokens, N = 256 hidden, K = 16),
+// accumulated in TMEM, and the epilogue applies b1, SiLU, w2 and b2 in fp32.
+//
+// split_weights_kernel writes Wh, Wl ([Hkv, 2, hidden, 3d] bf16) into the
+// workspace once per call.  score_kernel: one CTA = 256 tokens (two M = 128
+// accumulators, TMEM columns [0,256) and [256,512)) of one kv head; warp 8
+// streams B tiles (Wh, Wl of one 64-feature chunk, 2 x 32 KB, 2 stages) and
+// A tiles (128 tokens x 64 features of K, V or a q head, 16 KB, 4 stages)
+// with TMA; warp 9 issues the UMMAs; warps 0-7 run the epilogue, one token
+// row per thread.  Waits are bounded like the attention kernel's.
 #include <cuda_bf16.h>
 
 #include "apb_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace apb {
 namespace {
 
-constexpr int kTok = 64;        // tokens per CTA
-constexpr int kHid = 256;       // hidden units (all of them)
-constexpr int kChunk = 32;      // input features per shared-memory chunk
-constexpr int kXLd = kTok + 4;  // padded row of the transposed token chunk
-constexpr int kThreads = 256;
+constexpr int kHid = 256;
+constexpr int kTile = 128;                 // tokens per accumulator
+constexpr int kChunk = 64;                 // features per chunk (128-byte rows)
+constexpr int kAStages = 4;
+constexpr int kBStages = 2;
+constexpr int kATile = kTile * kChunk * 2;          // 16 KB
+constexpr int kBHalf = kHid * kChunk * 2;           // 32 KB (hi or lo)
+constexpr int kSmemA = 0;
+constexpr int kSmemB = kAStages * kATile;           // 64 KB
+constexpr int kSmemBars = kSmemB + kBStages * 2 * kBHalf;   // 192 KB
+constexpr int kSmemBytes = kSmemBars + 256 + 2 * kHid * 4 + 1024;
+constexpr int kThreads = 320;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 t = __bfloat1622float2(p[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
+enum Bar { A_FULL = 0, A_EMPTY = 4, B_FULL = 8, B_EMPTY = 10, ACC_FULL = 12, DRAIN = 13, NUM = 14 };
+
+__global__ void __launch_bounds__(256) split_weights_kernel(const float* __restrict__ w1,
+                                                            __nv_bfloat16* __restrict__ ws,
+                                                            int Hkv, int F, int d, int G) {
+  const long long per_head = (long long)kHid * F;
+  const long long total = (long long)Hkv * per_head;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long g = i / per_head;
+    const long long rem = i - g * per_head;
+    const int f = (int)(rem % F);
+    float w = w1[i];
+    if (f >= 2 * d) w = __fdiv_rn(w, (float)G);   // group mean folded in (exact for G = 2^k)
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+    ws[(2 * g) * per_head + rem] = hi;
+    ws[(2 * g + 1) * per_head + rem] = lo;
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 2) score_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, const float* __restrict__ w1,
-    const float* __restrict__ b1, const float* __restrict__ w2, const float* __restrict__ b2,
-    float* __restrict__ scores, long long N, int Hq, int Hkv, int d) {
-  __shared__ __align__(16) float xs[kChunk][kXLd];
-  __shared__ __align__(16) float ws[kChunk][kHid];
+struct ScoreParams {
+  long long N;
+  int Hq, Hkv, G, d, F, n_chunks;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+  float* scores;
+  DeviceStatus* status;
+};
 
+__device__ void record_failure(DeviceStatus* st, uint32_t where, uint32_t tile) {
+  if (atomicOr(&st->sticky, kErrWaitTimeout) == 0u) {
+    st->where = where;
+    st->tile = tile;
+  }
+  atomicExch(&st->abort, 1u);
+  __threadfence();
+}
+
+// A tiles of one chunk: 1 input block for k and v chunks, G for q chunks,
+// each for both 128-token halves.
+__device__ __forceinline__ int chunk_blocks(int c, int d, int G) {
+  return (c * kChunk) / d < 2 ? 1 : G;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    score_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                 const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mW,
+                 const ScoreParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBars);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + NUM);
+  uint32_t* s_flags = s_tmem + 1;
+  float* s_b1 = reinterpret_cast<float*>(smem + kSmemBars + 256);
+  float* s_w2 = s_b1 + kHid;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
-  const long long t0 = (long long)blockIdx.x * kTok;
-  const int G = Hq / Hkv;
-  const int F = 3 * d;
-  const int tid = threadIdx.x;
-  const int tg = tid >> 4;    // token group: tokens 4*tg .. 4*tg+3
-  const int hg = tid & 15;    // hidden group: units 4*hg + 64*i + j
-  const float* w1g = w1 + (long long)g * kHid * F;
+  const long long t0 = (long long)blockIdx.x * (2 * kTile);
+  const volatile uint32_t* gabort = &p.status->abort;
 
-  float acc[4][16];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 16; ++b) acc[a][b] = 0.f;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NUM; ++i) ptx::mbar_init(&bars[i], 1);
+    ptx::fence_mbar_init();
+    s_flags[0] = *gabort;
+    s_flags[1] = 0u;
+  }
+  if (threadIdx.x < kHid) {
+    s_b1[threadIdx.x] = p.b1[g * kHid + threadIdx.x];
+    s_w2[threadIdx.x] = p.w2[g * kHid + threadIdx.x];
+  }
+  if (warp == 9) {
+    ptx::tmem_alloc(s_tmem, 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    ptx::tma_prefetch_desc(&mQ);
+    ptx::tma_prefetch_desc(&mK);
+    ptx::tma_prefetch_desc(&mV);
+    ptx::tma_prefetch_desc(&mW);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const volatile uint32_t* never = s_flags + 1;
+  const bool skip = s_flags[0] != 0u;
 
-  // loader roles
-  const int ld_tok = tid >> 2;          // 0..63
-  const int ld_part = tid & 3;          // 8 features each
-  const long long ld_t = t0 + ld_tok;
-  const bool ld_ok = ld_t < N;
-  const float invG = 1.0f / (float)G;
-
-  for (int f0 = 0; f0 < F; f0 += kChunk) {
-    // ---- token chunk: features [f0, f0+32) of 64 tokens
-    {
-      const int sec = f0 / d;            // 0: k, 1: v, 2: mean q
-      const int off = f0 - sec * d + ld_part * 8;
-      float f[8];
-      if (!ld_ok) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.f;
-      } else if (sec < 2) {
-        const __nv_bfloat16* base = (sec == 0 ? k : v) + (ld_t * Hkv + g) * d + off;
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(base)), f);
-      } else {
-        float s8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.f;
-        for (int j = 0; j < G; ++j) {
-          const __nv_bfloat16* base = q + (ld_t * Hq + (long long)g * G + j) * d + off;
-          bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(base)), s8);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] += s8[i];
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !skip) {
+      int lastA[kAStages] = {-1, -1, -1, -1}, lastB[kBStages] = {-1, -1};
+      int ai = 0;
+      bool ok = true;
+      for (int c = 0; c < p.n_chunks && ok; ++c) {
+        const int bs = c & 1;
+        const uint32_t bpar = (c >> 1) & 1;
+        if (!ptx::mbar_wait_bounded(&bars[B_EMPTY + bs], bpar ^ 1, gabort, kWaitLimitNs)) {
+          record_failure(p.status, 70 + bs, c);
+          break;
         }
-        if ((G & (G - 1)) == 0) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] *= invG;
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = __fdiv_rn(f[i], (float)G);
+        uint8_t* bdst = smem + kSmemB + bs * 2 * kBHalf;
+        ptx::mbar_arrive_expect_tx(&bars[B_FULL + bs], 2 * kBHalf);
+        ptx::tma_load_3d(bdst, &mW, &bars[B_FULL + bs], c * kChunk, 0, 2 * g);
+        ptx::tma_load_3d(bdst + kBHalf, &mW, &bars[B_FULL + bs], c * kChunk, 0, 2 * g + 1);
+        lastB[bs] = (int)bpar;
+        const int sec = (c * kChunk) / p.d;
+        const int off = c * kChunk - sec * p.d;
+        const int nb = chunk_blocks(c, p.d, p.G);
+        for (int b = 0; b < nb && ok; ++b) {
+          for (int m = 0; m < 2; ++m, ++ai) {
+            const int as = ai % kAStages;
+            const uint32_t apar = (ai / kAStages) & 1;
+            if (!ptx::mbar_wait_bounded(&bars[A_EMPTY + as], apar ^ 1, gabort, kWaitLimitNs)) {
+              record_failure(p.status, 72, ai);
+              ok = false;
+              break;
+            }
+            uint8_t* adst = smem + kSmemA + as * kATile;
+            const int row = (int)(t0 + m * kTile);
+            ptx::mbar_arrive_expect_tx(&bars[A_FULL + as], kATile);
+            if (sec == 0)
+              ptx::tma_load_3d(adst, &mK, &bars[A_FULL + as], off, g, row);
+            else if (sec == 1)
+              ptx::tma_load_3d(adst, &mV, &bars[A_FULL + as], off, g, row);
+            else
+              ptx::tma_load_3d(adst, &mQ, &bars[A_FULL + as], off, g * p.G + b, row);
+            lastA[as] = (int)apar;
+          }
         }
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xs[ld_part * 8 + i][ld_tok] = f[i];
+      for (int s = 0; s < kAStages; ++s)
+        if (lastA[s] >= 0) ptx::mbar_wait_bounded(&bars[A_FULL + s], lastA[s], never, kWaitLimitNs);
+      for (int s = 0; s < kBStages; ++s)
+        if (lastB[s] >= 0) ptx::mbar_wait_bounded(&bars[B_FULL + s], lastB[s], never, kWaitLimitNs);
     }
-    // ---- W1 chunk: thread = hidden unit, 32 contiguous features, transposed
-    {
-      const float4* wrow = reinterpret_cast<const float4*>(w1g + (long long)tid * F + f0);
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && !skip) {
+      const uint32_t idesc = ptx::idesc_bf16_f32(kTile, kHid, 0);
+      const uint32_t aA = ptx::smem_u32(smem + kSmemA);
+      const uint32_t aB = ptx::smem_u32(smem + kSmemB);
+      bool started[2] = {false, false};
+      int ai = 0;
+      bool ok = true;
+      for (int c = 0; c < p.n_chunks && ok; ++c) {
+        const int bs = c & 1;
+        if (!ptx::mbar_wait_bounded(&bars[B_FULL + bs], (c >> 1) & 1, gabort, kWaitLimitNs)) {
+          record_failure(p.status, 74, c);
+          break;
+        }
+        ptx::tc_fence_after();
+        const int nb = chunk_blocks(c, p.d, p.G);
+        for (int b = 0; b < nb && ok; ++b) {
+          for (int m = 0; m < 2; ++m, ++ai) {
+            const int as = ai % kAStages;
+            if (!ptx::mbar_wait_bounded(&bars[A_FULL + as], (ai / kAStages) & 1, gabort,
+                                        kWaitLimitNs)) {
+              record_failure(p.status, 75, ai);
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < kChunk / 4; ++c) {
-        float4 w = __ldg(wrow + c);
-        ws[4 * c + 0][tid] = w.x;
-        ws[4 * c + 1][tid] = w.y;
-        ws[4 * c + 2][tid] = w.z;
-        ws[4 * c + 3][tid] = w.w;
+            for (int ks = 0; ks < kChunk / 16; ++ks) {
+#pragma unroll
+              for (int part = 0; part < 2; ++part) {
+                ptx::umma_bf16_ss(tmem + 256 * m,
+                                  ptx::sdesc_sw128(aA + as * kATile + ks * 32, 16, 1024),
+                                  ptx::sdesc_sw128(aB + bs * 2 * kBHalf + part * kBHalf + ks * 32,
+                                                   16, 1024),
+                                  idesc, started[m] ? 1u : 0u);
+                started[m] = true;
+              }
+            }
+            ptx::umma_commit(&bars[A_EMPTY + as]);
+          }
+        }
+        if (ok) ptx::umma_commit(&bars[B_EMPTY + bs]);
       }
+      if (ok) ptx::umma_commit(&bars[ACC_FULL]);
+      ptx::umma_commit(&bars[DRAIN]);
+      ptx::mbar_wait_bounded(&bars[DRAIN], 0, never, kWaitLimitNs);
     }
-    __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kChunk; ++kk) {
-      const float4 xa = *reinterpret_cast<const float4*>(&xs[kk][tg * 4]);
-      const float xr[4] = {xa.x, xa.y, xa.z, xa.w};
-      float wr[16];
+  } else if (!skip) {
+    // ------------------------------------------------------------ epilogue
+    const int m = warp >> 2;                        // token half
+    const int row = threadIdx.x & 127;
+    const uint32_t taddr = tmem + 256 * m + ((uint32_t)((warp & 3) * 32) << 16);
+    bool ok = ptx::mbar_wait_bounded(&bars[ACC_FULL], 0, gabort, kWaitLimitNs);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) record_failure(p.status, 76, m);
+    } else {
+      ptx::tc_fence_after();
+      float part = 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < kHid / 32; ++cc) {
+        uint32_t z[32];
+        APB_TMEM_LD32(taddr + 32 * cc, z);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 w = *reinterpret_cast<const float4*>(&ws[kk][hg * 4 + 64 * i]);
-        wr[4 * i + 0] = w.x;
-        wr[4 * i + 1] = w.y;
-        wr[4 * i + 2] = w.z;
-        wr[4 * i + 3] = w.w;
+        for (int x = 0; x < 32; ++x) {
+          const float zz = __uint_as_float(z[x]) + s_b1[32 * cc + x];
+          const float silu = __fdividef(zz, 1.0f + __expf(-zz));
+          part = fmaf(s_w2[32 * cc + x], silu, part);
+        }
       }
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 16; ++b) acc[a][b] = fmaf(xr[a], wr[b], acc[a][b]);
+      const long long t = t0 + m * kTile + row;
+      if (t < p.N) p.scores[(long long)g * p.N + t] = part + p.b2[g];
     }
-    __syncthreads();
   }
 
-  // ---- epilogue: b1, SiLU, w2, reduce over the 16 hidden groups
-  const float* b1g = b1 + (long long)g * kHid;
-  const float* w2g = w2 + (long long)g * kHid;
-  float bb[16], ww[16];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int u = hg * 4 + 64 * i + j;
-      bb[4 * i + j] = __ldg(b1g + u);
-      ww[4 * i + j] = __ldg(w2g + u);
-    }
-  const float bias2 = __ldg(b2 + g);
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    float part = 0.f;
-#pragma unroll
-    for (int b = 0; b < 16; ++b) {
-      const float z = acc[a][b] + bb[b];
-      const float silu = z / (1.0f + expf(-z));
-      part = fmaf(ww[b], silu, part);
-    }
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    const long long t = t0 + tg * 4 + a;
-    if (hg == 0 && t < N) scores[(long long)g * N + t] = part + bias2;
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -165,11 +271,49 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(
 
 cudaError_t launch_score(const Shape& s, const void* q, const void* k, const void* v,
                          const float* w1, const float* b1, const float* w2, const float* b2,
-                         float* scores, cudaStream_t st) {
-  dim3 grid((unsigned)((s.N + kTok - 1) / kTok), s.Hkv);
-  score_kernel<<<grid, kThreads, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), w1, b1, w2, b2, scores, s.N, s.Hq, s.Hkv, s.d);
+                         float* scores, void* wsplit, DeviceStatus* status, cudaStream_t st,
+                         const char** why) {
+  const int F = 3 * s.d;
+  const int G = s.Hq / s.Hkv;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  split_weights_kernel<<<sms * 4, 256, 0, st>>>(w1, static_cast<__nv_bfloat16*>(wsplit), s.Hkv,
+                                                F, s.d, G);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap mQ, mK, mV, mW;
+  const uint64_t N = (uint64_t)s.N;
+  bool ok = encode_bf16_3d(&mQ, q, s.d, s.Hq, N, (uint64_t)s.d * 2, (uint64_t)s.Hq * s.d * 2, 64,
+                           1, kTile) &&
+            encode_bf16_3d(&mK, k, s.d, s.Hkv, N, (uint64_t)s.d * 2, (uint64_t)s.Hkv * s.d * 2, 64,
+                           1, kTile) &&
+            encode_bf16_3d(&mV, v, s.d, s.Hkv, N, (uint64_t)s.d * 2, (uint64_t)s.Hkv * s.d * 2, 64,
+                           1, kTile) &&
+            encode_bf16_3d(&mW, wsplit, F, kHid, (uint64_t)s.Hkv * 2, (uint64_t)F * 2,
+                           (uint64_t)kHid * F * 2, 64, kHid, 1);
+  if (!ok) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point or argument)";
+    return cudaErrorInvalidValue;
+  }
+  ScoreParams p;
+  p.N = s.N;
+  p.Hq = s.Hq;
+  p.Hkv = s.Hkv;
+  p.G = G;
+  p.d = s.d;
+  p.F = F;
+  p.n_chunks = F / kChunk;
+  p.b1 = b1;
+  p.w2 = w2;
+  p.b2 = b2;
+  p.scores = scores;
+  p.status = status;
+  e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((s.N + 2 * kTile - 1) / (2 * kTile)), s.Hkv);
+  score_kernel<<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, mW, p);
   return cudaGetLastError();
 }
 

@@ -6,8 +6,9 @@
 // keeps in the caller's workspace live here in a fixed, file-scope device
 // array instead, so the call needs no workspace and allocates nothing.
 //
-// The array holds kStaticScoreFloats floats (16 MiB).  Every GPU that loads
-// this library reserves it until the process exits.
+// The arrays hold kStaticScoreFloats floats (16 MiB) for the scores and
+// kStaticWsBytes bytes (8 MiB + 256) for the status block and the bf16 split of
+// W1.  Every GPU that loads this library reserves them until the process exits.
 #include <mutex>
 
 #include "apb_internal.h"
@@ -15,17 +16,20 @@
 namespace {
 
 constexpr size_t kStaticScoreFloats = size_t(4) << 20;   // Hkv * N <= 4,194,304
+constexpr size_t kStaticWsBytes = 256 + (size_t(8) << 20);   // status + W1 split
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_score_scratch[kStaticScoreFloats];
+static __device__ __align__(256) unsigned char g_ws_scratch[kStaticWsBytes];
 
 std::mutex g_mutex;
 float* g_scratch_ptr[kMaxDevices] = {};
+void* g_ws_ptr[kMaxDevices] = {};
 
-// Device address of g_score_scratch on the current device.  In host code the
-// symbol is only a host-side handle, so the address must come from
-// cudaGetSymbolAddress, once per device, with that device current.
-cudaError_t scratch_address(float** out) {
+// Device addresses of the two arrays on the current device.  In host code a
+// __device__ symbol is only a host-side handle, so the addresses must come
+// from cudaGetSymbolAddress, once per device, with that device current.
+cudaError_t scratch_address(float** out, void** ws) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -33,11 +37,16 @@ cudaError_t scratch_address(float** out) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
+    void* w = nullptr;
     e = cudaGetSymbolAddress(&p, g_score_scratch);
     if (e != cudaSuccess) return e;
+    e = cudaGetSymbolAddress(&w, g_ws_scratch);
+    if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = static_cast<float*>(p);
+    g_ws_ptr[dev] = w;
   }
   *out = g_scratch_ptr[dev];
+  *ws = g_ws_ptr[dev];
   return cudaSuccess;
 }
 
@@ -55,17 +64,22 @@ apb_status apb_score_compress_static(const apb_config* cfg, const void* q, const
   if (apb_workspace_bytes(cfg) == 0)
     return apb_score_compress(cfg, q, k, v, w1, b1, w2, b2, nullptr, idx, nullptr, 0, stream);
   const size_t need = (size_t)cfg->n_kv_heads * (size_t)cfg->n_hosts * (size_t)cfg->block_len;
-  if (need > kStaticScoreFloats) return APB_ERR_UNSUPPORTED;
+  const size_t split = (size_t)cfg->n_kv_heads * 2 * cfg->mlp_hidden * 3 * cfg->head_dim * 2;
+  if (need > kStaticScoreFloats || 256 + ((split + 255) & ~size_t(255)) > kStaticWsBytes)
+    return APB_ERR_UNSUPPORTED;
   if (!q || !k || !v || !w1 || !b1 || !w2 || !b2 || (cfg->keep > 0 && !idx))
     return APB_ERR_INVALID_ARG;
   float* scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return APB_ERR_CUDA;
-  // The scratch takes the place of the caller-owned scores buffer: every
-  // score the top-k reads is written by this same call first, so nothing in
-  // it needs clearing.  With a scores buffer given, apb_score_compress never
-  // touches its workspace argument; the scratch address fills that slot.
-  return apb_score_compress(cfg, q, k, v, w1, b1, w2, b2, scratch, idx, scratch,
-                            apb::kStatusBytes, stream);
+  void* ws = nullptr;
+  if (scratch_address(&scratch, &ws) != cudaSuccess) return APB_ERR_CUDA;
+  // The arrays take the place of the caller's scores buffer and workspace.
+  // Every score and weight the kernels read is written by this same call
+  // first; the status block starts at zero (static storage) and its abort
+  // flag is cleared by every call, so nothing else needs clearing.  A bounded
+  // wait that runs out is recorded in this private status block, which no
+  // call reports.
+  return apb_score_compress(cfg, q, k, v, w1, b1, w2, b2, scratch, idx, ws, kStaticWsBytes,
+                            stream);
 }
 
 }  // extern "C"
