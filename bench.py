@@ -165,6 +165,11 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def rank_config(cfg, rank):
+    """Each rank prefills its own sequence: same workload, its own seed."""
+    return cfg.replace(seed=cfg.seed + 1000 * rank)
+
+
 def config_dict(cfg, world):
     return {"workload": cfg.name, "seq_len": cfg.seq_len, "n_hosts": cfg.n_hosts,
             "block_len": cfg.block_len, "anchor_len": cfg.anchor_len, "keep": cfg.keep,
@@ -250,7 +255,7 @@ def run_gpu(args, cfg):
 
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
-    rcfg = cfg.replace(seed=cfg.seed + 1000 * rank)     # independent sequence per rank
+    rcfg = rank_config(cfg, rank)                       # independent sequence per rank
     x = inputs.generate(rcfg)
     xd = {k: v.to(dev) for k, v in x.items() if k != "needles"}
     c = apb.make_config(rcfg)
@@ -335,6 +340,10 @@ def run_gpu(args, cfg):
     barrier(world)
     e2e_value = world * cfg.seq_len / (e2e_ms / 1e3 / e2e_steps)
 
+    variants = None
+    if not args.no_variants:
+        variants = attention_variants(apb, cfg, xd, dev, stream, attn_ms)
+
     if rank != 0:
         if world > 1:
             import torch.distributed as dist
@@ -378,6 +387,7 @@ def run_gpu(args, cfg):
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel runs "
                                     f"{attn_ms:.1f} ms per launch, back to back)"},
         "cpu_baseline": cpu,
+        "variants": variants,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (5 if cfg.keep > 0 else 3),
@@ -387,6 +397,32 @@ def run_gpu(args, cfg):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def attention_variants(apb, cfg, xd, dev, stream, apb_ms, reps=3):
+    """The same attention kernel on the same Q/K/V with the two masks the
+    pages compare APB against: dense causal attention over the whole
+    sequence (one host), and a Star-Attention-style pattern (anchor = a whole
+    block, no passing block).  Reports the APB mask's speed-up over each."""
+    out = {"apb_ms": apb_ms}
+    shapes = {"dense_causal": dict(n_hosts=1, block_len=cfg.seq_len, anchor_len=0, query_len=0,
+                                   keep=0),
+              "star": dict(anchor_len=cfg.block_len, keep=0)}
+    for name, kw in shapes.items():
+        c = apb.make_config(cfg, **kw)
+        apb.block_attention(c, xd["q"], xd["k"], xd["v"], None, None, out=None, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        o = torch.empty_like(xd["q"])
+        e0.record(stream)
+        for _ in range(reps):
+            apb.block_attention(c, xd["q"], xd["k"], xd["v"], None, None, out=o, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / reps
+        out[f"{name}_ms"] = ms
+        out[f"apb_speedup_vs_{name}"] = ms / apb_ms
+        del o
+    return out
 
 
 def apb_kernel_rev() -> str:
@@ -406,6 +442,8 @@ def main():
     ap.add_argument("--workload", default="llama8b_128k", choices=sorted(inputs.CONFIGS))
     ap.add_argument("--oracle-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the dense-causal and Star-style timings of the same kernel")
     args = ap.parse_args()
     cfg = inputs.CONFIGS[args.workload]
     if args.impl == "reference":

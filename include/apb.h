@@ -157,6 +157,18 @@ apb_status apb_score_compress_static(const apb_config* cfg, const void* q, const
                                      const float* w2, const float* b2, int32_t* idx,
                                      void* stream);
 
+/* No counterpart in the paper: a self-test of the bounded waits every kernel
+ * uses.  Launches two CTAs that each wait on an on-chip barrier that nothing
+ * completes: CTA 0 with a limit of limit_us microseconds (1..1000000), CTA 1
+ * with a limit 20 times longer plus 1 s.  CTA 0's wait runs out and records
+ * APB_ERR_TIMEOUT in the status block of `workspace` (>= 256 bytes, zeroed
+ * before first use); CTA 1 leaves its wait through the launch-wide abort
+ * flag.  Bytes 64..79 of the block receive the two waits' elapsed
+ * nanoseconds.  apb_device_status then reports APB_ERR_TIMEOUT.  Nothing
+ * faults, traps or hangs. */
+apb_status apb_selftest_wait_timeout(void* workspace, size_t ws_bytes, uint32_t limit_us,
+                                     void* stream);
+
 /* Synchronises `stream`, then reads the status block of `workspace`:
  * APB_ERR_TIMEOUT if a kernel recorded a bounded wait that ran out since the
  * block was last cleared, else APB_OK (APB_ERR_CUDA if the reads fail).

@@ -47,6 +47,8 @@ _lib.apb_score_compress_static.argtypes = [ctypes.POINTER(Config)] + [_P] * 9
 _lib.apb_score_compress_static.restype = ctypes.c_int
 _lib.apb_score_compress_static_max_floats.argtypes = []
 _lib.apb_score_compress_static_max_floats.restype = ctypes.c_size_t
+_lib.apb_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
+_lib.apb_selftest_wait_timeout.restype = ctypes.c_int
 _lib.apb_device_status.argtypes = [_P, _P, ctypes.c_int]
 _lib.apb_device_status.restype = ctypes.c_int
 _lib.apb_status_string.argtypes = [ctypes.c_int]
@@ -230,6 +232,16 @@ def block_attention(c: Config, q, k, v, pass_k, pass_v, out=None, lse=None, want
 def device_status(workspace, stream=None, clear=False) -> int:
     """apb_device_status: synchronises the stream, returns the status code."""
     return int(_lib.apb_device_status(_ptr(workspace), _stream(stream), 1 if clear else 0))
+
+
+def selftest_wait_timeout(workspace, limit_us: int, stream=None):
+    """apb_selftest_wait_timeout: two CTAs wait on barriers that nothing
+    completes; returns the launch status.  Read the outcome with
+    device_status(); the two waits' elapsed nanoseconds are bytes 64..79 of
+    the workspace."""
+    st = _lib.apb_selftest_wait_timeout(_ptr(workspace), workspace.numel(), limit_us,
+                                        _stream(stream))
+    _check(st, "apb_selftest_wait_timeout")
 
 
 class Prefill:

@@ -16,6 +16,8 @@ struct DeviceStatus {
   uint32_t where;      // role/barrier id of the first failed wait
   uint32_t tile;       // tile index of the first failed wait
 };
+// Bytes [64, 80) of the status block: elapsed times written by the wait
+// self-test; the rest of the 256 bytes is reserved.
 constexpr uint32_t kErrWaitTimeout = 1u;
 constexpr size_t kStatusBytes = 256;
 

@@ -37,6 +37,7 @@
 // drains its outstanding TMA loads and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 #include "apb_internal.h"
+#include "device_status.cuh"
 #include "sm100_ptx.cuh"
 
 namespace apb {
@@ -82,15 +83,6 @@ struct Params {
   float* lse;
   DeviceStatus* status;
 };
-
-__device__ void record_failure(DeviceStatus* st, uint32_t where, uint32_t tile) {
-  if (atomicOr(&st->sticky, kErrWaitTimeout) == 0u) {
-    st->where = where;
-    st->tile = tile;
-  }
-  atomicExch(&st->abort, 1u);
-  __threadfence();
-}
 
 template <int D>
 __device__ __forceinline__ void load_kv_tile(const CUtensorMap* m_kv, const CUtensorMap* m_pass,

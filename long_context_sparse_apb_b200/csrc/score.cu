@@ -26,6 +26,7 @@
 #include <cuda_bf16.h>
 
 #include "apb_internal.h"
+#include "device_status.cuh"
 #include "sm100_ptx.cuh"
 
 namespace apb {
@@ -75,15 +76,6 @@ struct ScoreParams {
   float* scores;
   DeviceStatus* status;
 };
-
-__device__ void record_failure(DeviceStatus* st, uint32_t where, uint32_t tile) {
-  if (atomicOr(&st->sticky, kErrWaitTimeout) == 0u) {
-    st->where = where;
-    st->tile = tile;
-  }
-  atomicExch(&st->abort, 1u);
-  __threadfence();
-}
 
 // A tiles of one chunk: 1 input block for k and v chunks, G for q chunks,
 // each for both 128-token halves.

@@ -92,3 +92,10 @@ def test_null_and_misaligned_pointers_rejected():
 def test_keep_zero_build_passing_is_a_no_op():
     c = apb.make_config(inputs.TINY, keep=0)
     assert apb._lib.apb_build_passing(ctypes.byref(c), None, None, None, None, None, None) == 0
+
+
+def test_selftest_argument_checks():
+    assert apb._lib.apb_selftest_wait_timeout(None, 256, 1000, None) == apb.APB_ERR_INVALID_ARG
+    assert apb._lib.apb_selftest_wait_timeout(FAKE, 64, 1000, None) == apb.APB_ERR_INVALID_ARG
+    assert apb._lib.apb_selftest_wait_timeout(FAKE, 256, 0, None) == apb.APB_ERR_INVALID_ARG
+    assert apb._lib.apb_selftest_wait_timeout(FAKE, 256, 2_000_000, None) == apb.APB_ERR_INVALID_ARG
