@@ -48,27 +48,38 @@ constexpr int kThreads = 320;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
+// Which pairs of every 8 take 2^x on the FMA pipe instead of MUFU ex2
+// (balances the two pipes; the rest use ex2.approx).
+#ifndef APB_POLY_OF_8
+#define APB_POLY_OF_8 0
+#endif
+__device__ constexpr bool kPolyPairs[8] = {
+    APB_POLY_OF_8 > 0, APB_POLY_OF_8 > 4, APB_POLY_OF_8 > 2, APB_POLY_OF_8 > 6,
+    APB_POLY_OF_8 > 1, APB_POLY_OF_8 > 5, APB_POLY_OF_8 > 3, APB_POLY_OF_8 > 7};
 
 enum Bar {
   Q_FULL = 0,
-  K_FULL = 1,    // 2 stages
-  K_EMPTY = 3,   // 2
-  V_FULL = 5,    // 2
-  V_EMPTY = 7,   // 2
-  S_FULL = 9,    // per query tile (A, B)
-  P_FULL = 11,   // per query tile
-  O_FINAL = 13,  // per query tile
-  DRAIN = 15,
-  NUM_BARS = 16
+  K_FULL = 1,    // kKStages
+  K_EMPTY = 3,   // kKStages
+  V_FULL = 5,    // kVStages
+  V_EMPTY = 8,   // kVStages
+  S_FULL = 11,   // per query tile (A, B)
+  P_FULL = 13,   // per query tile and 64-column half: 13 + 2 * tile + half
+  O_FINAL = 17,  // per query tile
+  DRAIN = 19,
+  NUM_BARS = 20
 };
+
+constexpr int kKStages = 2;
+constexpr int kVStages = 3;   // V is released later than K: one more stage of prefetch
 
 template <int D>
 struct Layout {
   static constexpr int kTile = kRows * D * 2;   // bytes of one Q/K/V tile
   static constexpr int kQ = 0;                  // Q_A, Q_B
   static constexpr int kK0 = 2 * kTile;         // K stages
-  static constexpr int kV0 = 4 * kTile;         // V stages
-  static constexpr int kBars = 6 * kTile;
+  static constexpr int kV0 = kK0 + kKStages * kTile;   // V stages
+  static constexpr int kBars = kV0 + kVStages * kTile;
   static constexpr int kBytes = kBars + 256;
 };
 // Both head sizes request the d = 128 footprint so that one CTA runs per SM
@@ -140,8 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM_BARS; ++i) ptx::mbar_init(&bars[i], 1);
-    ptx::mbar_init(&bars[P_FULL], 128);
-    ptx::mbar_init(&bars[P_FULL + 1], 128);
+    for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars[P_FULL + i], 128);
     ptx::fence_mbar_init();
     s_flags[0] = *gabort;
     s_flags[1] = 0u;
@@ -171,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !skip) {
-      int lastK[2] = {-1, -1}, lastV[2] = {-1, -1};   // parity of the last load per slot
+      int lastK[kKStages] = {-1, -1}, lastV[kVStages] = {-1, -1, -1};   // last load parity per slot
       ptx::mbar_arrive_expect_tx(&bars[Q_FULL], (TB > 0 ? 2 : 1) * L::kTile);
       for (int i = 0; i < (TB > 0 ? 2 : 1); ++i) {
 #pragma unroll
@@ -180,57 +190,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                            head, local_row0 + qA0 + i * kRows);
       }
       for (int j = 0; j < Tmax; ++j) {
-        const int s = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        if (!ptx::mbar_wait_bounded(&bars[K_EMPTY + s], par ^ 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 40 + s, j);
+        const int ks = j % kKStages, vs = j % kVStages;
+        const uint32_t kpar = (j / kKStages) & 1, vpar = (j / kVStages) & 1;
+        if (!ptx::mbar_wait_bounded(&bars[K_EMPTY + ks], kpar ^ 1, gabort, kWaitLimitNs)) {
+          record_failure(p.status, 40 + ks, j);
           break;
         }
-        ptx::mbar_arrive_expect_tx(&bars[K_FULL + s], L::kTile);
-        load_kv_tile<D>(&mK, &mPK, sK0 + s * L::kTile, &bars[K_FULL + s], j, na, np, g,
+        ptx::mbar_arrive_expect_tx(&bars[K_FULL + ks], L::kTile);
+        load_kv_tile<D>(&mK, &mPK, sK0 + ks * L::kTile, &bars[K_FULL + ks], j, na, np, g,
                         local_row0);
-        lastK[s] = (int)par;
-        if (!ptx::mbar_wait_bounded(&bars[V_EMPTY + s], par ^ 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 42 + s, j);
+        lastK[ks] = (int)kpar;
+        if (!ptx::mbar_wait_bounded(&bars[V_EMPTY + vs], vpar ^ 1, gabort, kWaitLimitNs)) {
+          record_failure(p.status, 42 + vs, j);
           break;
         }
-        ptx::mbar_arrive_expect_tx(&bars[V_FULL + s], L::kTile);
-        load_kv_tile<D>(&mV, &mPV, sV0 + s * L::kTile, &bars[V_FULL + s], j, na, np, g,
+        ptx::mbar_arrive_expect_tx(&bars[V_FULL + vs], L::kTile);
+        load_kv_tile<D>(&mV, &mPV, sV0 + vs * L::kTile, &bars[V_FULL + vs], j, na, np, g,
                         local_row0);
-        lastV[s] = (int)par;
+        lastV[vs] = (int)vpar;
       }
       // drain: every load issued must have landed before the CTA exits
       ptx::mbar_wait_bounded(&bars[Q_FULL], 0, never, kWaitLimitNs);
-      for (int s = 0; s < 2; ++s) {
+      for (int s = 0; s < kKStages; ++s)
         if (lastK[s] >= 0) ptx::mbar_wait_bounded(&bars[K_FULL + s], lastK[s], never, kWaitLimitNs);
+      for (int s = 0; s < kVStages; ++s)
         if (lastV[s] >= 0) ptx::mbar_wait_bounded(&bars[V_FULL + s], lastV[s], never, kWaitLimitNs);
-      }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && !skip) {
       const uint32_t idesc_s = ptx::idesc_bf16_f32(kRows, kRows, 0);
       const uint32_t idesc_pv = ptx::idesc_bf16_f32(kRows, D, 1);
-      const uint32_t aQ = ptx::smem_u32(sQ);
-      const uint32_t aK0 = ptx::smem_u32(sK0), aV0 = ptx::smem_u32(sV0);
+      // Descriptors of the first K step of every operand buffer; a K step
+      // (or a stage) moves only the start-address field (bits 0-13, in
+      // 16-byte units), so each UMMA needs one add.
+      const uint64_t dQ = ptx::sdesc_sw128(ptx::smem_u32(sQ), 16, 1024);
+      const uint64_t dK = ptx::sdesc_sw128(ptx::smem_u32(sK0), 16, 1024);
+      const uint64_t dV = ptx::sdesc_sw128(ptx::smem_u32(sV0), kRows * 128, 1024);
+      constexpr uint32_t kTile16 = L::kTile >> 4;
       const int T[2] = {TA, TB};
 
       // S_i(jj) = Q_i K(jj)^T into S_i; K(jj) must have landed
       auto issue_s = [&](int i, int jj) {
-        const int s = jj & 1;
+        const uint64_t q = dQ + i * kTile16;
+        const uint64_t k = dK + (jj % kKStages) * kTile16;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
-          ptx::umma_bf16_ss(tmem + 128 * i, ptx::sdesc_sw128(aQ + i * L::kTile + off, 16, 1024),
-                            ptx::sdesc_sw128(aK0 + s * L::kTile + off, 16, 1024), idesc_s,
-                            kk > 0);
+          const uint32_t off = ((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4;
+          ptx::umma_bf16_ss(tmem + 128 * i, q + off, k + off, idesc_s, kk > 0);
         }
         ptx::umma_commit(&bars[S_FULL + i]);
       };
       auto wait_k = [&](int jj) -> bool {
-        if (!ptx::mbar_wait_bounded(&bars[K_FULL + (jj & 1)], (jj >> 1) & 1, gabort,
+        if (!ptx::mbar_spin_bounded(&bars[K_FULL + jj % kKStages], (jj / kKStages) & 1, gabort,
                                     kWaitLimitNs)) {
-          record_failure(p.status, 51 + (jj & 1), jj);
+          record_failure(p.status, 51 + jj % kKStages, jj);
           return false;
         }
         ptx::tc_fence_after();
@@ -243,11 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         issue_s(0, 0);
         if (TB > 0) issue_s(1, 0);
-        ptx::umma_commit(&bars[K_EMPTY]);
+        ptx::umma_commit(&bars[K_EMPTY + 0]);
       }
       for (int j = 0; ok && j < Tmax; ++j) {
-        const int s = j & 1;
-        if (!ptx::mbar_wait_bounded(&bars[V_FULL + s], (j >> 1) & 1, gabort, kWaitLimitNs)) {
+        const int s = j % kVStages;
+        if (!ptx::mbar_spin_bounded(&bars[V_FULL + s], (j / kVStages) & 1, gabort, kWaitLimitNs)) {
           record_failure(p.status, 54 + s, j);
           break;
         }
@@ -255,18 +269,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool k_next = false;   // K(j+1) waited for
         for (int i = 0; i < 2 && ok; ++i) {
           if (j >= T[i]) continue;
-          if (!ptx::mbar_wait_bounded(&bars[P_FULL + i], j & 1, gabort, kWaitLimitNs)) {
-            record_failure(p.status, 56 + i, j);
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
           const uint32_t tP = tmem + 128 * i;
+          const uint64_t v = dV + s * kTile16;
+          // P_i(j) arrives in two 64-column halves; PV on the first half
+          // overlaps the softmax's exponentials of the second
+          for (int half = 0; half < 2 && ok; ++half) {
+            if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i + half], j & 1, gabort,
+                                        kWaitLimitNs)) {
+              record_failure(p.status, 56 + 2 * i + half, j);
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk)
-            ptx::umma_bf16_ts(tmem + 256 + 128 * i, tP + kk * 8,
-                              ptx::sdesc_sw128(aV0 + s * L::kTile + kk * 2048, kRows * 128, 1024),
-                              idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = half * 4 + k4;
+              ptx::umma_bf16_ts(tmem + 256 + 128 * i, tP + kk * 8, v + ((kk * 2048) >> 4),
+                                idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          // V(j)'s last reader is PV_B(j) (or PV_A(j) when tile B has no tile j):
+          // release its slot now, before the next S MMA, so its reload starts early
+          if (i == 1 || j >= T[1]) ptx::umma_commit(&bars[V_EMPTY + s]);
           if (j + 1 < T[i]) {
             if (!k_next) {
               if (!(ok = wait_k(j + 1))) break;
@@ -278,8 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        ptx::umma_commit(&bars[V_EMPTY + s]);
-        if (k_next) ptx::umma_commit(&bars[K_EMPTY + ((j + 1) & 1)]);
+        if (k_next) ptx::umma_commit(&bars[K_EMPTY + (j + 1) % kKStages]);
       }
       // drain every MMA issued so far
       ptx::umma_commit(&bars[DRAIN]);
@@ -322,11 +346,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float mx[8];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) mx[x] = __uint_as_float(sr[x]);
+      for (int x = 0; x < 8; ++x)
+        mx[x] = fmaxf(__uint_as_float(sr[2 * x]), __uint_as_float(sr[2 * x + 1]));
 #pragma unroll
-      for (int c = 8; c < kRows; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
-      const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int c = 16; c < kRows; c += 2)
+        mx[(c >> 1) & 7] = ptx::fmax3(mx[(c >> 1) & 7], __uint_as_float(sr[c]),
+                                      __uint_as_float(sr[c + 1]));
+      const float tmax = fmaxf(ptx::fmax3(mx[0], mx[1], mx[2]),
+                               fmaxf(ptx::fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_tile = tmax * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -339,31 +366,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale = true;
       }
       const float mneg = -m;
-      uint32_t pk[64];
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, mneg));
-        const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, mneg));
-        sum[c & 3] += p0 + p1;
-        pk[c] = ptx::pack_bf16x2(p0, p1);
+      for (int half = 0; half < 2; ++half) {
+        if (half == 1) {
+          // reload the second half of S (cheaper than keeping 64 more
+          // registers alive through the first half)
+          APB_TMEM_LD32(tS + 64, sr + 64);
+          APB_TMEM_LD32(tS + 96, sr + 96);
+          if (lim < kRows) {
+#pragma unroll
+            for (int c = 64; c < kRows; ++c)
+              if (c >= lim) sr[c] = 0xff800000u;   // -inf
+          }
+        }
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          const int c = half * 32 + cc;
+          float x0, x1, p0, p1;
+          ptx::ffma2_scalar(x0, x1, __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]),
+                            p.scale_log2, mneg);
+          if (kPolyPairs[cc & 7]) {
+            ptx::exp2_poly2(p0, p1, x0, x1);      // part of the pairs on the FMA pipe
+          } else {
+            p0 = ptx::ex2(x0);
+            p1 = ptx::ex2(x1);
+          }
+          ptx::fadd2_acc(sum[(c & 1) * 2], sum[(c & 1) * 2 + 1], p0, p1);
+          pk[cc] = ptx::pack_bf16x2(p0, p1);
+        }
+        // O_i is stable here (the commit that signalled S_i(j) covers
+        // PV_i(j-1)); it must be rescaled before PV_i(j) starts on half 0
+        if (half == 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            APB_TMEM_LD32(tO + 32 * c, o);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            APB_TMEM_ST32(tO + 32 * c, o);
+          }
+        }
+        APB_TMEM_ST32(tS + 32 * half, pk);
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars[P_FULL + 2 * i + half]);
       }
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
-      // O_i is stable here: the commit that signalled S_i(j) covers PV_i(j-1)
-      if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          APB_TMEM_LD32(tO + 32 * c, o);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-          APB_TMEM_ST32(tO + 32 * c, o);
-        }
-      }
-      APB_TMEM_ST64(tS, pk);
-      ptx::tmem_st_wait();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars[P_FULL + i]);
     }
     if (ok && T > 0) {
       ok = ptx::mbar_wait_bounded(&bars[O_FINAL + i], 0, gabort, kWaitLimitNs);

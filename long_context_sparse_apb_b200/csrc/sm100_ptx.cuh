@@ -52,6 +52,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Like mbar_wait_bounded below, but polls without suspending the thread, for
+// the single thread whose reaction time is on the critical path (the UMMA
+// issuer): it sees the phase flip within a few cycles instead of after a
+// suspend/wake round trip.
+__device__ __forceinline__ bool mbar_spin_bounded(uint64_t* bar, uint32_t parity,
+                                                  const volatile uint32_t* abort,
+                                                  uint64_t limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+      if (mbar_test_wait(a, parity)) return true;
+    if (*abort != 0u) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
+  }
+}
+
 // Waits for the phase of parity `parity` of `bar` to complete.  Gives up and
 // returns false when `limit_ns` of wall time pass, or when *abort (a flag in
 // global memory that another CTA of the launch may set) becomes non-zero.
@@ -160,11 +191,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
       "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"         \
       "tcgen05.wait::ld.sync.aligned;"                                                           \
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),      \
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),  \
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),            \
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),            \
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])             \
+      : "=r"((r)[0]), "=r"((r)[1]), "=r"((r)[2]), "=r"((r)[3]), "=r"((r)[4]), "=r"((r)[5]), "=r"((r)[6]),      \
+        "=r"((r)[7]), "=r"((r)[8]), "=r"((r)[9]), "=r"((r)[10]), "=r"((r)[11]), "=r"((r)[12]), "=r"((r)[13]),  \
+        "=r"((r)[14]), "=r"((r)[15]), "=r"((r)[16]), "=r"((r)[17]), "=r"((r)[18]), "=r"((r)[19]),            \
+        "=r"((r)[20]), "=r"((r)[21]), "=r"((r)[22]), "=r"((r)[23]), "=r"((r)[24]), "=r"((r)[25]),            \
+        "=r"((r)[26]), "=r"((r)[27]), "=r"((r)[28]), "=r"((r)[29]), "=r"((r)[30]), "=r"((r)[31])             \
       : "r"(taddr)                                                                               \
       : "memory")
 
@@ -172,11 +203,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
   asm volatile(                                                                                  \
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13," \
       "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr), \
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),    \
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),          \
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),        \
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),        \
-      "r"(r[29]), "r"(r[30]), "r"(r[31])                                                         \
+      "r"((r)[0]), "r"((r)[1]), "r"((r)[2]), "r"((r)[3]), "r"((r)[4]), "r"((r)[5]), "r"((r)[6]), "r"((r)[7]),    \
+      "r"((r)[8]), "r"((r)[9]), "r"((r)[10]), "r"((r)[11]), "r"((r)[12]), "r"((r)[13]), "r"((r)[14]),          \
+      "r"((r)[15]), "r"((r)[16]), "r"((r)[17]), "r"((r)[18]), "r"((r)[19]), "r"((r)[20]), "r"((r)[21]),        \
+      "r"((r)[22]), "r"((r)[23]), "r"((r)[24]), "r"((r)[25]), "r"((r)[26]), "r"((r)[27]), "r"((r)[28]),        \
+      "r"((r)[29]), "r"((r)[30]), "r"((r)[31])                                                         \
       : "memory")
 
 // 32 lanes x 128 consecutive 32-bit columns (one full 128-column S tile per
@@ -185,7 +216,7 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
   asm volatile(                                                              \
       "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t" \
       "tcgen05.wait::ld.sync.aligned;"                                       \
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])                                                             \
+      : "=r"((r)[0]), "=r"((r)[1]), "=r"((r)[2]), "=r"((r)[3]), "=r"((r)[4]), "=r"((r)[5]), "=r"((r)[6]), "=r"((r)[7]), "=r"((r)[8]), "=r"((r)[9]), "=r"((r)[10]), "=r"((r)[11]), "=r"((r)[12]), "=r"((r)[13]), "=r"((r)[14]), "=r"((r)[15]), "=r"((r)[16]), "=r"((r)[17]), "=r"((r)[18]), "=r"((r)[19]), "=r"((r)[20]), "=r"((r)[21]), "=r"((r)[22]), "=r"((r)[23]), "=r"((r)[24]), "=r"((r)[25]), "=r"((r)[26]), "=r"((r)[27]), "=r"((r)[28]), "=r"((r)[29]), "=r"((r)[30]), "=r"((r)[31]), "=r"((r)[32]), "=r"((r)[33]), "=r"((r)[34]), "=r"((r)[35]), "=r"((r)[36]), "=r"((r)[37]), "=r"((r)[38]), "=r"((r)[39]), "=r"((r)[40]), "=r"((r)[41]), "=r"((r)[42]), "=r"((r)[43]), "=r"((r)[44]), "=r"((r)[45]), "=r"((r)[46]), "=r"((r)[47]), "=r"((r)[48]), "=r"((r)[49]), "=r"((r)[50]), "=r"((r)[51]), "=r"((r)[52]), "=r"((r)[53]), "=r"((r)[54]), "=r"((r)[55]), "=r"((r)[56]), "=r"((r)[57]), "=r"((r)[58]), "=r"((r)[59]), "=r"((r)[60]), "=r"((r)[61]), "=r"((r)[62]), "=r"((r)[63]), "=r"((r)[64]), "=r"((r)[65]), "=r"((r)[66]), "=r"((r)[67]), "=r"((r)[68]), "=r"((r)[69]), "=r"((r)[70]), "=r"((r)[71]), "=r"((r)[72]), "=r"((r)[73]), "=r"((r)[74]), "=r"((r)[75]), "=r"((r)[76]), "=r"((r)[77]), "=r"((r)[78]), "=r"((r)[79]), "=r"((r)[80]), "=r"((r)[81]), "=r"((r)[82]), "=r"((r)[83]), "=r"((r)[84]), "=r"((r)[85]), "=r"((r)[86]), "=r"((r)[87]), "=r"((r)[88]), "=r"((r)[89]), "=r"((r)[90]), "=r"((r)[91]), "=r"((r)[92]), "=r"((r)[93]), "=r"((r)[94]), "=r"((r)[95]), "=r"((r)[96]), "=r"((r)[97]), "=r"((r)[98]), "=r"((r)[99]), "=r"((r)[100]), "=r"((r)[101]), "=r"((r)[102]), "=r"((r)[103]), "=r"((r)[104]), "=r"((r)[105]), "=r"((r)[106]), "=r"((r)[107]), "=r"((r)[108]), "=r"((r)[109]), "=r"((r)[110]), "=r"((r)[111]), "=r"((r)[112]), "=r"((r)[113]), "=r"((r)[114]), "=r"((r)[115]), "=r"((r)[116]), "=r"((r)[117]), "=r"((r)[118]), "=r"((r)[119]), "=r"((r)[120]), "=r"((r)[121]), "=r"((r)[122]), "=r"((r)[123]), "=r"((r)[124]), "=r"((r)[125]), "=r"((r)[126]), "=r"((r)[127])                                                             \
       : "r"(taddr)                                                           \
       : "memory")
 
@@ -193,7 +224,7 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
 #define APB_TMEM_ST64(taddr, r)                                               \
   asm volatile(                                                              \
       "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};"        \
-      :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])                                                 \
+      :: "r"(taddr), "r"((r)[0]), "r"((r)[1]), "r"((r)[2]), "r"((r)[3]), "r"((r)[4]), "r"((r)[5]), "r"((r)[6]), "r"((r)[7]), "r"((r)[8]), "r"((r)[9]), "r"((r)[10]), "r"((r)[11]), "r"((r)[12]), "r"((r)[13]), "r"((r)[14]), "r"((r)[15]), "r"((r)[16]), "r"((r)[17]), "r"((r)[18]), "r"((r)[19]), "r"((r)[20]), "r"((r)[21]), "r"((r)[22]), "r"((r)[23]), "r"((r)[24]), "r"((r)[25]), "r"((r)[26]), "r"((r)[27]), "r"((r)[28]), "r"((r)[29]), "r"((r)[30]), "r"((r)[31]), "r"((r)[32]), "r"((r)[33]), "r"((r)[34]), "r"((r)[35]), "r"((r)[36]), "r"((r)[37]), "r"((r)[38]), "r"((r)[39]), "r"((r)[40]), "r"((r)[41]), "r"((r)[42]), "r"((r)[43]), "r"((r)[44]), "r"((r)[45]), "r"((r)[46]), "r"((r)[47]), "r"((r)[48]), "r"((r)[49]), "r"((r)[50]), "r"((r)[51]), "r"((r)[52]), "r"((r)[53]), "r"((r)[54]), "r"((r)[55]), "r"((r)[56]), "r"((r)[57]), "r"((r)[58]), "r"((r)[59]), "r"((r)[60]), "r"((r)[61]), "r"((r)[62]), "r"((r)[63])                                                 \
       : "memory")
 
 // D[tmem] (+)= A[tmem] * B[smem], kind::f16: A (M x 16 per instruction) is
@@ -223,6 +254,75 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ---------------------------------------------------------------- packed fp32
+// (x0, x1) * (a, a) + (b, b) as one packed f32x2 FMA.
+__device__ __forceinline__ void ffma2_scalar(float& y0, float& y1, float x0, float x1, float a,
+                                             float b) {
+  asm("{\n\t.reg .b64 u, v, w, r;\n\t"
+      "mov.b64 u, {%2, %3};\n\t"
+      "mov.b64 v, {%4, %4};\n\t"
+      "mov.b64 w, {%5, %5};\n\t"
+      "fma.rn.f32x2 r, u, v, w;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(a), "f"(b));
+}
+
+// (acc0, acc1) += (x0, x1) as one packed f32x2 add.
+__device__ __forceinline__ void fadd2_acc(float& acc0, float& acc1, float x0, float x1) {
+  asm("{\n\t.reg .b64 u, v;\n\t"
+      "mov.b64 u, {%0, %1};\n\t"
+      "mov.b64 v, {%2, %3};\n\t"
+      "add.rn.f32x2 u, u, v;\n\t"
+      "mov.b64 {%0, %1}, u;\n\t}"
+      : "+f"(acc0), "+f"(acc1)
+      : "f"(x0), "f"(x1));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe (no MUFU): Cody-Waite style reduction
+// x = n + f with n = rint(x) (magic-number rounding), f in [-1/2, 1/2], then
+// 2^f by a degree-3 polynomial fitted here by iteratively reweighted least
+// squares on Chebyshev nodes (max relative error 7.5e-5, below the 2^-9
+// rounding of the bf16 probabilities it feeds), and 2^n added to the
+// exponent field.  x is clamped to >= -125 so the result stays a positive
+// normal number (2^-125 stands for 0 next to row sums >= 1).
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
+  constexpr float c2 = 0.2426111251115799f, c3 = 0.05517164617776871f;
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  uint32_t t0b, t1b, p0b, p1b;
+  asm("{\n\t.reg .b64 x, t, n, f, p, m, mn, k;\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "mov.b64 m, {%6, %6};\n\t"
+      "mov.b64 mn, {%7, %7};\n\t"
+      "add.rn.f32x2 t, x, m;\n\t"            // t = x + magic (integer n in low bits)
+      "add.rn.f32x2 n, t, mn;\n\t"           // n = rint(x)
+      "mov.b64 k, {%12, %12};\n\t"
+      "fma.rn.f32x2 f, n, k, x;\n\t"         // f = x - n
+      "mov.b64 p, {%11, %11};\n\t"
+      "mov.b64 k, {%10, %10};\n\t"
+      "fma.rn.f32x2 p, p, f, k;\n\t"         // c3 f + c2
+      "mov.b64 k, {%9, %9};\n\t"
+      "fma.rn.f32x2 p, p, f, k;\n\t"         // (.) f + c1
+      "mov.b64 k, {%8, %8};\n\t"
+      "fma.rn.f32x2 p, p, f, k;\n\t"         // (.) f + c0
+      "mov.b64 {%0, %1}, t;\n\t"
+      "mov.b64 {%2, %3}, p;\n\t}"
+      : "=r"(t0b), "=r"(t1b), "=r"(p0b), "=r"(p1b)
+      : "f"(x0), "f"(x1), "f"(kMagic), "f"(-kMagic), "f"(c0), "f"(c1), "f"(c2), "f"(c3),
+        "f"(-1.0f));
+  y0 = __uint_as_float(p0b + (t0b << 23));
+  y1 = __uint_as_float(p1b + (t1b << 23));
 }
 
 }  // namespace ptx
