@@ -266,3 +266,67 @@ class Prefill:
         block_attention(self.c, q, k, v, self.pass_k, self.pass_v, out=self.out,
                         workspace=self.workspace, stream=stream)
         return self.out
+
+
+class PrefillPipeline:
+    """Prefills of successive sequences from pinned host memory with the
+    transfers of one step overlapped with the compute of another.
+
+    Each of `depth` slots owns device copies of the inputs and a Prefill
+    (workspace, indices, passing block, output).  submit() queues, on three
+    streams ordered by events, the host->device copy of the step's inputs,
+    the three calls of the path, and the device->host copy of the output into
+    the caller's pinned buffer.  A slot's inputs are overwritten only after its
+    previous compute has finished, and its output only after the previous copy
+    back has finished.  synchronize() waits for everything queued."""
+
+    def __init__(self, c: Config, device="cuda", depth: int = 2):
+        N, hq, hkv, d = _dims(c)
+        dev = torch.device(device)
+        self.c = c
+        self.depth = depth
+        self.h2d = torch.cuda.Stream(dev)
+        self.comp = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.slots = []
+        for _ in range(depth):
+            x = {"q": torch.empty((N, hq, d), dtype=torch.bfloat16, device=dev),
+                 "k": torch.empty((N, hkv, d), dtype=torch.bfloat16, device=dev),
+                 "v": torch.empty((N, hkv, d), dtype=torch.bfloat16, device=dev),
+                 "w1": torch.empty((hkv, c.mlp_hidden, 3 * d), dtype=torch.float32, device=dev),
+                 "b1": torch.empty((hkv, c.mlp_hidden), dtype=torch.float32, device=dev),
+                 "w2": torch.empty((hkv, c.mlp_hidden), dtype=torch.float32, device=dev),
+                 "b2": torch.empty((hkv,), dtype=torch.float32, device=dev)}
+            ev = {k: torch.cuda.Event() for k in ("in", "comp", "out")}
+            self.slots.append({"x": x, "run": Prefill(c, device=dev), "ev": ev, "used": False})
+        self.i = 0
+
+    def submit(self, host: dict, host_out: torch.Tensor) -> None:
+        """host: pinned CPU tensors q, k, v, w1, b1, w2, b2; host_out: pinned
+        CPU bf16 [N, Hq, d] receiving this step's output."""
+        slot = self.slots[self.i % self.depth]
+        self.i += 1
+        ev = slot["ev"]
+        with torch.cuda.stream(self.h2d):
+            if slot["used"]:
+                self.h2d.wait_event(ev["comp"])          # previous compute done reading
+            for k, t in slot["x"].items():
+                t.copy_(host[k], non_blocking=True)
+            ev["in"].record(self.h2d)
+        with torch.cuda.stream(self.comp):
+            self.comp.wait_event(ev["in"])
+            if slot["used"]:
+                self.comp.wait_event(ev["out"])          # previous output copied back
+            x = slot["x"]
+            slot["run"](x["q"], x["k"], x["v"], x["w1"], x["b1"], x["w2"], x["b2"],
+                        stream=self.comp)
+            ev["comp"].record(self.comp)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(ev["comp"])
+            host_out.copy_(slot["run"].out, non_blocking=True)
+            ev["out"].record(self.d2h)
+        slot["used"] = True
+
+    def synchronize(self) -> None:
+        for st in (self.h2d, self.comp, self.d2h):
+            st.synchronize()

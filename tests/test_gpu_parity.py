@@ -129,3 +129,27 @@ def test_dense_causal_reduction_on_gpu(apb):
     ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)[0]
     err = (out.float().permute(1, 0, 2) - ref).abs()
     assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3
+
+
+def test_pipeline_matches_direct_calls(apb):
+    # PrefillPipeline (pinned host buffers, overlapped copies) returns, for
+    # each submitted step, exactly what the direct calls return
+    cfgs = [inputs.TINY, inputs.TINY.replace(seed=5)]
+    xs = [inputs.generate(c) for c in cfgs]
+    c = apb.make_config(inputs.TINY)
+    direct = []
+    for x in xs:
+        xd = _to_dev(x)
+        run = apb.Prefill(c)
+        direct.append(run(xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"], xd["b2"]).cpu())
+    pipe = apb.PrefillPipeline(c, depth=2)
+    outs = []
+    for step in range(5):
+        x = xs[step % 2]
+        hx = {k: v.pin_memory() for k, v in x.items() if k != "needles"}
+        ho = torch.empty_like(direct[0]).pin_memory()
+        pipe.submit(hx, ho)
+        outs.append((step % 2, ho, hx))
+    pipe.synchronize()
+    for which, ho, _ in outs:
+        assert torch.equal(ho, direct[which])
