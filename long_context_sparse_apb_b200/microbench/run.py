@@ -1,4 +1,5 @@
-"""Builds and runs the UMMA-rate microbenchmark (umma_rate.cu) on cuda:0.
+"""Builds and runs the UMMA-rate microbenchmarks (umma_rate.cu, single SM;
+umma_pair_rate.cu, cta_group::2 pairs) on cuda:0.
 
     python -m long_context_sparse_apb_b200.microbench.run
 """
@@ -11,12 +12,15 @@ ROOT = os.path.dirname(os.path.dirname(HERE))
 
 
 def main() -> int:
-    exe = os.path.join(ROOT, "_build", "umma_rate")
-    os.makedirs(os.path.dirname(exe), exist_ok=True)
-    subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
-                    "-I", os.path.join(ROOT, "include"), os.path.join(HERE, "umma_rate.cu"), "-o",
-                    exe], check=True)
-    return subprocess.run([exe]).returncode
+    rc = 0
+    for name in ("umma_rate", "umma_pair_rate"):
+        exe = os.path.join(ROOT, "_build", name)
+        os.makedirs(os.path.dirname(exe), exist_ok=True)
+        subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
+                        "-I", os.path.join(ROOT, "include"), os.path.join(HERE, name + ".cu"),
+                        "-o", exe], check=True)
+        rc |= subprocess.run([exe]).returncode
+    return rc
 
 
 if __name__ == "__main__":
