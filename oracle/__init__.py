@@ -3,8 +3,8 @@
 Only the test suite, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU
 baseline leg may import this package.
 """
-from .apb_oracle import (retaining_scores, compress_indices, passing_blocks,
+from .apb_oracle import (retaining_scores, retaining_scores_query_aware, compress_indices, passing_blocks,
                          host_attention, visible_pairs)
 
-__all__ = ["retaining_scores", "compress_indices", "passing_blocks",
+__all__ = ["retaining_scores", "retaining_scores_query_aware", "compress_indices", "passing_blocks",
            "host_attention", "visible_pairs"]

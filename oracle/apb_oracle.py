@@ -31,6 +31,8 @@ Readings taken where the pages are silent:
       concat(k[t,g], v[t,g], mean over the group's q heads of q[t,j]) through
       Linear(3d, hidden) -> SiLU -> Linear(hidden, 1);
   R6  q head j uses kv head j // G (consecutive grouping);
+  R5b (query-aware variant) the q part of the MLP input is the mean of the
+      query segment over its rows and the group's q heads, for every token;
   R7  top-k ties: the lower position wins; indices are returned ascending.
 
 Every function below is checked by ``tests/test_oracle_pins.py`` against
@@ -70,6 +72,38 @@ def retaining_scores(q, k, v, w1, b1, w2, b2):
         for g in range(hkv):
             x = np.concatenate([k[:, g, :], v[:, g, :], qbar[:, g, :]], axis=1)
             z = x @ w1[g].T + b1[g]                        # [T, hidden]
+            a = z / (1.0 + np.exp(-z))
+            s[g] = a @ w2[g] + b2[g]
+    return s
+
+
+def retaining_scores_query_aware(q_seg, k, v, w1, b1, w2, b2):
+    """Query-aware variant of the stand-in score ("APB 的技术原理": the query is
+    embedded at the start of the anchor so that the compressor sees it).
+
+    Reading R5b: the q part of the MLP input is the mean of the query segment
+    (rows [0, q_len) of the sequence) over its rows and over the group's q
+    heads, the same for every token:
+        qseg[g] = mean_{r < q_len, j: j//G == g} q[r, j]     (0 if q_len == 0)
+        x = [k[t,g] ; v[t,g] ; qseg[g]],   s[g,t] as in retaining_scores.
+
+    q_seg [q_len, Hq, d] (the query segment), k/v [T, Hkv, d], weights as in
+    retaining_scores.  Returns s [Hkv, T] float64.
+    """
+    q_seg, k, v = _f64(q_seg), _f64(k), _f64(v)
+    w1, b1, w2, b2 = _f64(w1), _f64(b1), _f64(w2), _f64(b2)
+    T, hkv, d = k.shape
+    L, hq, _ = q_seg.shape
+    G = hq // hkv
+    if L > 0:
+        qm = q_seg.reshape(L, hkv, G, d).mean(axis=(0, 2))   # [Hkv, d]
+    else:
+        qm = np.zeros((hkv, d))
+    s = np.empty((hkv, T), dtype=F64)
+    with np.errstate(over="ignore"):
+        for g in range(hkv):
+            x = np.concatenate([k[:, g, :], v[:, g, :], np.broadcast_to(qm[g], (T, d))], axis=1)
+            z = x @ w1[g].T + b1[g]
             a = z / (1.0 + np.exp(-z))
             s[g] = a @ w2[g] + b2[g]
     return s

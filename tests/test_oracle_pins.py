@@ -22,7 +22,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (compress_indices, host_attention, passing_blocks,
+from oracle import (compress_indices, host_attention, passing_blocks, retaining_scores_query_aware,
                     retaining_scores, visible_pairs)
 from long_context_sparse_apb_b200 import inputs
 
@@ -300,3 +300,37 @@ def test_anchor_fraction_matches_pages():
         assert cfg.anchor_len / cfg.block_len in g["allowed_fractions"], cfg.name
         assert 0 <= cfg.query_len <= cfg.anchor_len <= cfg.block_len
         assert cfg.n_q_heads % cfg.n_kv_heads == 0
+
+
+# ----------------------------------------------------------------- query-aware score
+
+def test_query_aware_equals_own_token_score_when_q_is_the_segment():
+    # if every token's q equals one fixed row and the segment holds that row,
+    # the two readings of the q input coincide
+    T, hq, hkv, d = 7, 4, 2, 8
+    row = _rand((1, hq, d), 30)
+    q = np.repeat(row, T, axis=0)
+    k, v = _rand((T, hkv, d), 31), _rand((T, hkv, d), 32)
+    w1, b1 = _rand((hkv, 16, 3 * d), 33, 0.1), _rand((hkv, 16), 34, 0.1)
+    w2, b2 = _rand((hkv, 16), 35, 0.1), _rand((hkv,), 36, 0.1)
+    a = retaining_scores(q, k, v, w1, b1, w2, b2)
+    b = retaining_scores_query_aware(np.repeat(row, 3, axis=0), k, v, w1, b1, w2, b2)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-14)
+
+
+def test_query_aware_closed_form_and_empty_segment():
+    from oracle import retaining_scores_query_aware as qa
+    ln3 = math.log(3.0)
+    # d = 1, G = 2: segment rows q = (2, 4) and (0, 2) -> mean 2; hidden unit = qseg * ln3/2
+    q_seg = np.array([[[2.0], [4.0]], [[0.0], [2.0]]])
+    k = np.array([[[5.0]], [[-1.0]]])
+    v = np.zeros((2, 1, 1))
+    w1 = np.array([[[0.0, 0.0, ln3 / 2], [1.0, 0.0, 0.0]]])   # unit0 = ln3 (qseg), unit1 = k
+    b1 = np.zeros((1, 2))
+    w2 = np.array([[4.0, 0.0]])
+    b2 = np.array([0.5])
+    s = qa(q_seg, k, v, w1, b1, w2, b2)
+    np.testing.assert_allclose(s[0], [4 * 0.75 * ln3 + 0.5] * 2, atol=1e-14)   # SiLU(ln3) = 3/4 ln3
+    # empty segment: q part is zero
+    s0 = qa(np.zeros((0, 2, 1)), k, v, w1, b1, w2, b2)
+    np.testing.assert_allclose(s0[0], [0.5, 0.5], atol=1e-14)
