@@ -412,7 +412,8 @@ def attention_variants(apb, cfg, xd, dev, stream, apb_ms, reps=3):
     """The same attention kernel on the same Q/K/V with the two masks the
     pages compare APB against: dense causal attention over the whole
     sequence (one host), and a Star-Attention-style pattern (anchor = a whole
-    block, no passing block).  Reports the APB mask's speed-up over each."""
+    block, no passing block).  Reports the APB mask's speed-up over each, and
+    the score + top-k time of the query-aware compression variant."""
     out = {"apb_ms": apb_ms}
     shapes = {"dense_causal": dict(n_hosts=1, block_len=cfg.seq_len, anchor_len=0, query_len=0,
                                    keep=0),
@@ -431,6 +432,20 @@ def attention_variants(apb, cfg, xd, dev, stream, apb_ms, reps=3):
         out[f"{name}_ms"] = ms
         out[f"apb_speedup_vs_{name}"] = ms / apb_ms
         del o
+    # query-aware compression (q input = query-segment mean): score + top-k time
+    c = apb.make_config(cfg)
+    ws = apb.new_workspace(c)
+    w = (xd["w1"], xd["b1"], xd["w2"], xd["b2"])
+    apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, workspace=ws, stream=stream,
+                       query_aware=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, workspace=ws, stream=stream,
+                           query_aware=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    out["query_aware_score_topk_ms"] = e0.elapsed_time(e1) / reps
     return out
 
 

@@ -77,8 +77,9 @@ typedef struct apb_config {
 
 /* Bytes of device workspace that apb_score_compress and apb_block_attention
  * need: a 256-byte status block, then the bf16 hi/lo split of W1
- * (Hkv*hidden*3d*4 bytes, rounded up to 256), then Hkv*N*4 bytes (rounded up
- * to 256) for the scores when apb_score_compress is given scores == NULL.
+ * (Hkv*hidden*3d*4 bytes, rounded up to 256), then the query-aware bias
+ * (Hkv*hidden*4 bytes, rounded up to 256), then Hkv*N*4 bytes (rounded up to
+ * 256) for the scores when a score call is given scores == NULL.
  * Returns 0 for a NULL or invalid config.  The caller zero-fills a workspace
  * once before its first use (the status block must start at zero). */
 size_t apb_workspace_bytes(const apb_config* cfg);
@@ -104,6 +105,24 @@ apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* 
                               const float* w2, const float* b2, float* scores,
                               int32_t* idx, void* workspace, size_t ws_bytes,
                               void* stream);
+
+/* Step 1, query-aware variant (technical principles: the query is embedded
+ * at the start of the anchor so the compressor sees it and keeps the KV pairs
+ * that matter for it).  Same arguments, outputs and selection rule as
+ * apb_score_compress, but the q part of the MLP input is, for every token,
+ * the mean of q over the query segment (rows [0, query_len)) and the group's
+ * q heads (zero when query_len == 0):
+ *     x = [k[t,g] ; v[t,g] ; mean_{r < q_len, j: j/G == g} q[r,j]]
+ * That part is constant per kv head, so it is folded exactly into the first
+ * layer's bias (fp32) and the product runs over the k and v sections only;
+ * Q rows beyond the query segment are not read.  The workspace additionally
+ * holds that bias (Hkv*hidden*4 bytes): apb_workspace_bytes(cfg) bytes, or,
+ * when scores is given, the status block, the weight split and the bias. */
+apb_status apb_score_compress_query_aware(const apb_config* cfg, const void* q, const void* k,
+                                          const void* v, const float* w1, const float* b1,
+                                          const float* w2, const float* b2, float* scores,
+                                          int32_t* idx, void* workspace, size_t ws_bytes,
+                                          void* stream);
 
 /* Step 2 (main features: communication; the all-gather of compressed blocks
  * and the passing block built from the preceding hosts' blocks).

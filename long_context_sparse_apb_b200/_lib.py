@@ -39,6 +39,8 @@ _lib.apb_workspace_bytes.argtypes = [ctypes.POINTER(Config)]
 _lib.apb_workspace_bytes.restype = ctypes.c_size_t
 _lib.apb_score_compress.argtypes = [ctypes.POINTER(Config)] + [_P] * 10 + [ctypes.c_size_t, _P]
 _lib.apb_score_compress.restype = ctypes.c_int
+_lib.apb_score_compress_query_aware.argtypes = _lib.apb_score_compress.argtypes
+_lib.apb_score_compress_query_aware.restype = ctypes.c_int
 _lib.apb_build_passing.argtypes = [ctypes.POINTER(Config)] + [_P] * 6
 _lib.apb_build_passing.restype = ctypes.c_int
 _lib.apb_block_attention.argtypes = [ctypes.POINTER(Config)] + [_P] * 8 + [ctypes.c_size_t, _P]
@@ -133,8 +135,9 @@ def new_workspace(c: Config, device="cuda") -> torch.Tensor:
 
 
 def score_compress(c: Config, q, k, v, w1, b1, w2, b2, scores=None, idx=None, workspace=None,
-                   stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """apb_score_compress: returns (idx [H, Hkv, keep] int32, scores or None)."""
+                   stream=None, query_aware=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """apb_score_compress (or apb_score_compress_query_aware when
+    query_aware): returns (idx [H, Hkv, keep] int32, scores or None)."""
     N, hq, hkv, d = _dims(c)
     _want(q, "q", torch.bfloat16, (N, hq, d))
     _want(k, "k", torch.bfloat16, (N, hkv, d))
@@ -150,11 +153,11 @@ def score_compress(c: Config, q, k, v, w1, b1, w2, b2, scores=None, idx=None, wo
     _want(idx, "idx", torch.int32, (c.n_hosts, hkv, c.keep))
     if workspace is None:
         workspace = new_workspace(c, q.device)
-    st = _lib.apb_score_compress(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1),
-                                 _ptr(w2), _ptr(b2), _ptr(scores),
-                                 _ptr(idx) if idx.numel() else None, _ptr(workspace),
-                                 workspace.numel(), _stream(stream))
-    _check(st, "apb_score_compress")
+    fn = _lib.apb_score_compress_query_aware if query_aware else _lib.apb_score_compress
+    st = fn(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2),
+            _ptr(scores), _ptr(idx) if idx.numel() else None, _ptr(workspace), workspace.numel(),
+            _stream(stream))
+    _check(st, "apb_score_compress_query_aware" if query_aware else "apb_score_compress")
     return idx, scores
 
 

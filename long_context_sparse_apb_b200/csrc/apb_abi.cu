@@ -48,6 +48,7 @@ apb_status check_config(const apb_config* c, apb::Shape* s) {
   s->H = c->n_hosts;
   s->n = c->block_len;
   s->A = c->anchor_len;
+  s->ql = c->query_len;
   s->keep = c->keep;
   s->Hq = c->n_q_heads;
   s->Hkv = c->n_kv_heads;
@@ -72,35 +73,42 @@ size_t apb_workspace_bytes(const apb_config* cfg) {
   apb::Shape s;
   if (check_config(cfg, &s) != APB_OK) return 0;
   return apb::kStatusBytes + round256(apb::weight_split_bytes(s)) +
-         round256((size_t)s.Hkv * (size_t)s.N * sizeof(float));
+         round256(apb::query_bias_bytes(s)) + round256((size_t)s.Hkv * (size_t)s.N * sizeof(float));
 }
 
-apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* k,
-                              const void* v, const float* w1, const float* b1,
-                              const float* w2, const float* b2, float* scores,
-                              int32_t* idx, void* workspace, size_t ws_bytes,
-                              void* stream) {
+}  // extern "C"
+
+namespace {
+
+apb_status score_compress_impl(const char* who, bool query_aware, const apb_config* cfg,
+                               const void* q, const void* k, const void* v, const float* w1,
+                               const float* b1, const float* w2, const float* b2, float* scores,
+                               int32_t* idx, void* workspace, size_t ws_bytes, void* stream) {
   apb::Shape s;
   apb_status st = check_config(cfg, &s);
   if (st != APB_OK) return st;
   if (!q || !k || !v || !w1 || !b1 || !w2 || !b2 || !workspace)
-    return fail(APB_ERR_INVALID_ARG, "apb_score_compress: NULL input or workspace");
-  if (s.keep > 0 && !idx) return fail(APB_ERR_INVALID_ARG, "apb_score_compress: idx is NULL");
+    return fail(APB_ERR_INVALID_ARG, "%s: NULL input or workspace", who);
+  if (s.keep > 0 && !idx) return fail(APB_ERR_INVALID_ARG, "%s: idx is NULL", who);
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w1) || !aligned16(workspace) ||
       (scores && !aligned16(scores)) || (idx && !aligned16(idx)))
-    return fail(APB_ERR_INVALID_ARG, "apb_score_compress: pointers must be 16-byte aligned");
+    return fail(APB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
   const size_t wsplit = round256(apb::weight_split_bytes(s));
-  const size_t need = scores ? apb::kStatusBytes + wsplit : apb_workspace_bytes(cfg);
+  const size_t qbias = round256(apb::query_bias_bytes(s));
+  const size_t need = scores ? apb::kStatusBytes + wsplit + (query_aware ? qbias : 0)
+                             : apb_workspace_bytes(cfg);
   if (ws_bytes < need)
-    return fail(APB_ERR_INVALID_ARG, "apb_score_compress: workspace %zu < %zu bytes", ws_bytes, need);
+    return fail(APB_ERR_INVALID_ARG, "%s: workspace %zu < %zu bytes", who, ws_bytes, need);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   auto* status = reinterpret_cast<apb::DeviceStatus*>(ws);
-  float* sc = scores ? scores : reinterpret_cast<float*>(ws + apb::kStatusBytes + wsplit);
+  float* sc = scores ? scores : reinterpret_cast<float*>(ws + apb::kStatusBytes + wsplit + qbias);
+  float* qb = query_aware ? reinterpret_cast<float*>(ws + apb::kStatusBytes + wsplit) : nullptr;
   cudaError_t e = cudaMemsetAsync(&status->abort, 0, sizeof(uint32_t), cs);
   if (e != cudaSuccess) return cuda_fail(e, "clearing abort flag");
   const char* why = nullptr;
-  e = apb::launch_score(s, q, k, v, w1, b1, w2, b2, sc, ws + apb::kStatusBytes, status, cs, &why);
+  e = apb::launch_score(s, q, k, v, w1, b1, w2, b2, sc, ws + apb::kStatusBytes, qb, status, cs,
+                        &why);
   if (why) return fail(APB_ERR_CUDA, "score: %s", why);
   if (e != cudaSuccess) return cuda_fail(e, "score kernel");
   if (s.keep > 0) {
@@ -108,6 +116,29 @@ apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* 
     if (e != cudaSuccess) return cuda_fail(e, "top-k kernel");
   }
   return APB_OK;
+}
+
+
+}  // namespace
+
+extern "C" {
+
+apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* k,
+                              const void* v, const float* w1, const float* b1,
+                              const float* w2, const float* b2, float* scores,
+                              int32_t* idx, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  return score_compress_impl("apb_score_compress", false, cfg, q, k, v, w1, b1, w2, b2, scores,
+                             idx, workspace, ws_bytes, stream);
+}
+
+apb_status apb_score_compress_query_aware(const apb_config* cfg, const void* q, const void* k,
+                                          const void* v, const float* w1, const float* b1,
+                                          const float* w2, const float* b2, float* scores,
+                                          int32_t* idx, void* workspace, size_t ws_bytes,
+                                          void* stream) {
+  return score_compress_impl("apb_score_compress_query_aware", true, cfg, q, k, v, w1, b1, w2, b2,
+                             scores, idx, workspace, ws_bytes, stream);
 }
 
 apb_status apb_build_passing(const apb_config* cfg, const void* k, const void* v,

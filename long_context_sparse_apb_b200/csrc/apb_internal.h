@@ -22,7 +22,7 @@ constexpr uint32_t kErrWaitTimeout = 1u;
 constexpr size_t kStatusBytes = 256;
 
 struct Shape {
-  int H, n, A, keep, Hq, Hkv, d, hidden;
+  int H, n, A, ql, keep, Hq, Hkv, d, hidden;
   long long N;
   float scale;
 };
@@ -36,11 +36,17 @@ bool encode_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, 
 inline size_t weight_split_bytes(const Shape& s) {
   return (size_t)s.Hkv * 2 * s.hidden * 3 * s.d * 2;
 }
+// Bytes of the folded first-layer bias of the query-aware score variant.
+inline size_t query_bias_bytes(const Shape& s) { return (size_t)s.Hkv * s.hidden * 4; }
 
+// qbias == nullptr: the retaining-score stand-in on each token's own q.
+// qbias != nullptr: the query-aware variant; the query segment's mean q is
+// folded into a first-layer bias written to qbias ([Hkv, hidden] fp32) and
+// the q section of the product is skipped.
 cudaError_t launch_score(const Shape& s, const void* q, const void* k, const void* v,
                          const float* w1, const float* b1, const float* w2,
-                         const float* b2, float* scores, void* wsplit, DeviceStatus* status,
-                         cudaStream_t st, const char** why);
+                         const float* b2, float* scores, void* wsplit, float* qbias,
+                         DeviceStatus* status, cudaStream_t st, const char** why);
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* idx, cudaStream_t st);
 cudaError_t launch_gather(const Shape& s, const void* k, const void* v, const int32_t* idx,
                           void* pass_k, void* pass_v, cudaStream_t st);

@@ -67,6 +67,35 @@ __global__ void __launch_bounds__(256) split_weights_kernel(const float* __restr
   }
 }
 
+// Query-aware variant: the q input of the MLP is the same for every token,
+// qseg[g] = mean of q over the query segment rows [0, q_len) and the group's
+// G heads, so its product folds into the first-layer bias:
+//     qbias[g, u] = b1[g, u] + sum_f W1[g, u, 2d + f] * qseg[g, f]
+// One CTA per kv head; fp32 sums (q_len * G bf16 terms, then d products).
+__global__ void __launch_bounds__(256) query_bias_kernel(const __nv_bfloat16* __restrict__ q,
+                                                         const float* __restrict__ w1,
+                                                         const float* __restrict__ b1,
+                                                         float* __restrict__ qbias, int ql, int Hq,
+                                                         int G, int d) {
+  __shared__ float qm[128];
+  const int g = blockIdx.x;
+  const int F = 3 * d;
+  for (int f = threadIdx.x; f < d; f += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < ql; ++r)
+      for (int j = 0; j < G; ++j)
+        acc += __bfloat162float(q[((long long)r * Hq + (long long)g * G + j) * d + f]);
+    qm[f] = ql > 0 ? __fdiv_rn(acc, (float)(ql * G)) : 0.f;
+  }
+  __syncthreads();
+  for (int u = threadIdx.x; u < kHid; u += blockDim.x) {
+    const float* wrow = w1 + ((long long)g * kHid + u) * F + 2 * d;
+    float z = b1[g * kHid + u];
+    for (int f = 0; f < d; ++f) z = fmaf(wrow[f], qm[f], z);
+    qbias[g * kHid + u] = z;
+  }
+}
+
 struct ScoreParams {
   long long N;
   int Hq, Hkv, G, d, F, n_chunks;
@@ -263,8 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_score(const Shape& s, const void* q, const void* k, const void* v,
                          const float* w1, const float* b1, const float* w2, const float* b2,
-                         float* scores, void* wsplit, DeviceStatus* status, cudaStream_t st,
-                         const char** why) {
+                         float* scores, void* wsplit, float* qbias, DeviceStatus* status,
+                         cudaStream_t st, const char** why) {
   const int F = 3 * s.d;
   const int G = s.Hq / s.Hkv;
   int dev = 0, sms = 148;
@@ -274,6 +303,13 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
                                                 F, s.d, G);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+
+  if (qbias) {
+    query_bias_kernel<<<s.Hkv, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), w1, b1, qbias,
+                                             s.ql, s.Hq, G, s.d);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
 
   CUtensorMap mQ, mK, mV, mW;
   const uint64_t N = (uint64_t)s.N;
@@ -296,8 +332,10 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
   p.G = G;
   p.d = s.d;
   p.F = F;
-  p.n_chunks = F / kChunk;
-  p.b1 = b1;
+  // the query-aware variant stops after the k and v sections: its q section
+  // is a per-head constant already folded into qbias
+  p.n_chunks = (qbias ? 2 * s.d : F) / kChunk;
+  p.b1 = qbias ? qbias : b1;
   p.w2 = w2;
   p.b2 = b2;
   p.scores = scores;

@@ -71,3 +71,16 @@ def compare_attention(o_gpu: np.ndarray, o_ref: np.ndarray, what: str):
     mx, mean = float(err.max()), float(err.mean())
     assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, f"{what}: max {mx:.3e} mean {mean:.3e}"
     return mx, mean
+
+
+def oracle_scores_query_aware(cfg: inputs.APBConfig, x) -> np.ndarray:
+    """fp64 oracle of the query-aware score variant [Hkv, N]."""
+    n = cfg.block_len
+    out = np.empty((cfg.n_kv_heads, cfg.seq_len), dtype=np.float64)
+    w = [x[k].numpy() for k in ("w1", "b1", "w2", "b2")]
+    q_seg = f32np(x["q"][:cfg.query_len])
+    for h in range(cfg.n_hosts):
+        sl = slice(h * n, (h + 1) * n)
+        out[:, sl] = oracle.retaining_scores_query_aware(q_seg, f32np(x["k"][sl]),
+                                                         f32np(x["v"][sl]), *w)
+    return out

@@ -32,7 +32,7 @@ def test_status_strings():
 
 def test_workspace_bytes():
     c = apb.make_config(inputs.LLAMA8B_128K)
-    assert apb.workspace_bytes(c) == 256 + 8 * 256 * 384 * 4 + 8 * 131072 * 4
+    assert apb.workspace_bytes(c) == 256 + 8 * 256 * 384 * 4 + 8 * 256 * 4 + 8 * 131072 * 4
     bad = apb.make_config(inputs.TINY, keep=10_000)
     assert apb.workspace_bytes(bad) == 0
     assert apb._lib.apb_workspace_bytes(None) == 0

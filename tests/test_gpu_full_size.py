@@ -73,3 +73,21 @@ def test_full_size_workload(apb, name):
                                             cfg.anchor_len, cfg.keep, heads=heads)
         got = o_gpu_h[torch.as_tensor(rows, device=out.device)][:, heads].float().cpu().numpy()
         compare_attention(got, o_ref, f"{name} h{h} sample")
+
+
+@pytest.mark.parametrize("name", ["llama8b_32k", "llama8b_128k"])
+def test_full_size_query_aware_selection(apb, name):
+    from _parity import oracle_scores_query_aware
+    cfg = inputs.CONFIGS[name]
+    x = inputs.generate(cfg)
+    xd = {k: v.cuda() for k, v in x.items() if k != "needles"}
+    c = apb.make_config(cfg)
+    scores = torch.empty((cfg.n_kv_heads, cfg.seq_len), dtype=torch.float32, device="cuda")
+    ws = apb.new_workspace(c)
+    idx, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"],
+                                xd["b2"], scores=scores, workspace=ws, query_aware=True)
+    torch.cuda.synchronize()
+    assert apb.device_status(ws) == apb.APB_OK
+    s_ref = oracle_scores_query_aware(cfg, x)
+    assert np.abs(scores.cpu().numpy() - s_ref).max() <= SCORE_ABS
+    check_topk(idx.cpu().numpy(), s_ref, cfg)

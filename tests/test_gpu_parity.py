@@ -153,3 +153,29 @@ def test_pipeline_matches_direct_calls(apb):
     pipe.synchronize()
     for which, ho, _ in outs:
         assert torch.equal(ho, direct[which])
+
+
+@pytest.mark.parametrize("cfg", [inputs.TINY,
+                                 inputs.TINY.replace(n_hosts=3, block_len=300, anchor_len=75,
+                                                     query_len=0, keep=40, seed=9),
+                                 inputs.TINY.replace(n_q_heads=10, n_kv_heads=2, head_dim=128,
+                                                     seed=12)],
+                         ids=["tiny", "no_query_segment", "g5_d128"])
+def test_query_aware_scores_and_selection(apb, cfg):
+    from _parity import oracle_scores_query_aware
+    x = inputs.generate(cfg)
+    xd = _to_dev(x)
+    c = apb.make_config(cfg)
+    scores = torch.empty((cfg.n_kv_heads, cfg.seq_len), dtype=torch.float32, device="cuda")
+    ws = apb.new_workspace(c)
+    idx, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"],
+                                xd["b2"], scores=scores, workspace=ws, query_aware=True)
+    torch.cuda.synchronize()
+    assert apb.device_status(ws) == apb.APB_OK
+    s_ref = oracle_scores_query_aware(cfg, x)
+    assert np.abs(scores.cpu().numpy() - s_ref).max() <= SCORE_ABS
+    check_topk(idx.cpu().numpy(), s_ref, cfg)
+    # the two variants differ (own-token q vs query-segment q) unless q_len covers nothing
+    idx2, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"],
+                                 xd["b2"], workspace=ws)
+    assert idx2.shape == idx.shape
