@@ -415,23 +415,35 @@ def attention_variants(apb, cfg, xd, dev, stream, apb_ms, reps=3):
     block, no passing block).  Reports the APB mask's speed-up over each, and
     the score + top-k time of the query-aware compression variant."""
     out = {"apb_ms": apb_ms}
+    other_anchor = cfg.block_len // 4 if cfg.anchor_len * 8 == cfg.block_len else cfg.block_len // 8
     shapes = {"dense_causal": dict(n_hosts=1, block_len=cfg.seq_len, anchor_len=0, query_len=0,
                                    keep=0),
-              "star": dict(anchor_len=cfg.block_len, keep=0)}
+              "star": dict(anchor_len=cfg.block_len, keep=0),
+              # the pages' other anchor size (1/4 <-> 1/8 of a block), same keep
+              f"anchor_{other_anchor}": dict(anchor_len=other_anchor,
+                                             query_len=min(cfg.query_len, other_anchor))}
     for name, kw in shapes.items():
         c = apb.make_config(cfg, **kw)
-        apb.block_attention(c, xd["q"], xd["k"], xd["v"], None, None, out=None, stream=stream)
+        pk = pv = None
+        if c.keep > 0 and c.n_hosts > 1:
+            # the same compressed blocks as the APB step (the anchor size does not enter them)
+            run = apb.Prefill(c, device=dev)
+            apb.score_compress(c, xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"],
+                               xd["b2"], idx=run.idx, workspace=run.workspace, stream=stream)
+            pk, pv = apb.build_passing(c, xd["k"], xd["v"], run.idx, run.pass_k, run.pass_v,
+                                       stream=stream)
+        apb.block_attention(c, xd["q"], xd["k"], xd["v"], pk, pv, out=None, stream=stream)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         o = torch.empty_like(xd["q"])
         e0.record(stream)
         for _ in range(reps):
-            apb.block_attention(c, xd["q"], xd["k"], xd["v"], None, None, out=o, stream=stream)
+            apb.block_attention(c, xd["q"], xd["k"], xd["v"], pk, pv, out=o, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         ms = e0.elapsed_time(e1) / reps
         out[f"{name}_ms"] = ms
         out[f"apb_speedup_vs_{name}"] = ms / apb_ms
-        del o
+        del o, pk, pv
     # query-aware compression (q input = query-segment mean): score + top-k time
     c = apb.make_config(cfg)
     ws = apb.new_workspace(c)
@@ -449,6 +461,78 @@ def attention_variants(apb, cfg, xd, dev, stream, apb_ms, reps=3):
     return out
 
 
+def run_sharded(args, cfg):
+    """One sequence prefilled by N GPUs, hosts split evenly (the pages'
+    distributed form): per step each rank compresses its hosts, the compressed
+    blocks are all-gathered over NCCL, each rank attends its hosts.  Strong
+    scaling: value = tokens of the one sequence / max-over-ranks step time."""
+    from long_context_sparse_apb_b200 import _lib as apb
+    from long_context_sparse_apb_b200.sharded import ShardedPrefill, nccl_all_gather
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    c = apb.make_config(cfg)
+    sp = ShardedPrefill(c, rank, world, device=dev,
+                        all_gather=nccl_all_gather() if world > 1 else None)
+    loc = {k: v.to(dev) for k, v in inputs.generate_local(cfg, sp.hb, sp.he).items()}
+    w = (loc["w1"], loc["b1"], loc["w2"], loc["b2"])
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        sp.compress(loc["q"], loc["k"], loc["v"], *w)
+        if e is not None:
+            e[1].record(stream)
+        sp.exchange()
+        if e is not None:
+            e[2].record(stream)
+        sp.attend(loc["q"], loc["k"], loc["v"])
+        if e is not None:
+            e[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    if apb.device_status(sp.workspace) != apb.APB_OK:
+        raise RuntimeError("device status not OK after timed steps")
+    max_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    stages = {name: max_over_ranks(statistics.mean(e[a].elapsed_time(e[b]) for e in ev), world)
+              for name, a, b in (("compress", 0, 1), ("exchange", 1, 2), ("attention", 2, 3))}
+    if rank == 0:
+        cdict = config_dict(cfg, world)
+        cdict["parallelism"] = (f"host-sharded: {world} GPU(s) x {cfg.n_hosts // world} host(s), "
+                                f"NCCL all-gather of the compressed blocks")
+        line = {"metric": METRIC, "value": cfg.seq_len / (max_ms / 1e3 / args.steps),
+                "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": cdict, "stages_ms_max_over_ranks": stages,
+                "exchange_bytes_per_rank": 2 * (sp.he - sp.hb) * cfg.keep * cfg.n_kv_heads
+                * cfg.head_dim * 2,
+                "e2e": None, "e2e_note": "host-buffer end-to-end is measured in the default mode",
+                "gpu_launches": args.steps * (cfg.n_hosts // world) * (4 if cfg.keep else 2)
+                + args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def apb_kernel_rev() -> str:
     """Hash of the attention kernel source: ncu traffic counters only apply to
     the revision they were taken on."""
@@ -463,6 +547,10 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded"],
+                    help="replicas: one independent sequence per GPU (weak scaling); "
+                         "sharded: one sequence with its hosts split over the GPUs and an "
+                         "NCCL all-gather of the compressed blocks (strong scaling)")
     ap.add_argument("--workload", default="llama8b_128k", choices=sorted(inputs.CONFIGS))
     ap.add_argument("--oracle-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -472,6 +560,8 @@ def main():
     cfg = inputs.CONFIGS[args.workload]
     if args.impl == "reference":
         run_reference(args, cfg)
+    elif args.mode == "sharded":
+        run_sharded(args, cfg)
     else:
         run_gpu(args, cfg)
 

@@ -126,10 +126,14 @@ apb_status apb_score_compress_query_aware(const apb_config* cfg, const void* q, 
 
 /* Step 2 (main features: communication; the all-gather of compressed blocks
  * and the passing block built from the preceding hosts' blocks).
- *   pass_k[g, h*keep + r, :] = k[idx[h, g, r], g, :]   (and likewise v)
- *   pass_k, pass_v [Hkv, H*keep, d] bf16 (out), copied bit-exactly.
- * Host h's passing block is rows [0, h*keep) of this layout.  An index
- * outside [0, N) yields a zero row instead of a read. */
+ *   pass_k[h*keep + r, g, :] = k[idx[h, g, r], g, :]   (and likewise v)
+ *   pass_k, pass_v [H*keep, Hkv, d] bf16 (out, token-major like k and v),
+ *   copied bit-exactly.
+ * Host h's passing block is rows [0, h*keep) of this layout, and the blocks
+ * of hosts [a, b) are the contiguous rows [a*keep, b*keep): what one
+ * all-gather exchanges when hosts live on different GPUs.  idx may hold
+ * positions relative to the k/v pointers given (e.g. one host's block).  An
+ * index outside [0, N) yields a zero row instead of a read. */
 apb_status apb_build_passing(const apb_config* cfg, const void* k, const void* v,
                              const int32_t* idx, void* pass_k, void* pass_v,
                              void* stream);
@@ -148,6 +152,25 @@ apb_status apb_block_attention(const apb_config* cfg, const void* q, const void*
                                const void* v, const void* pass_k, const void* pass_v,
                                void* out, float* lse, void* workspace, size_t ws_bytes,
                                void* stream);
+
+/* Step 3 for a range of hosts on rank-local buffers (main features: the
+ * sequence is split over hosts, each host's context block is preceded by the
+ * anchor block, and the passing block is built from the all-gathered
+ * compressed blocks).  Computes exactly what apb_block_attention computes
+ * for hosts [host_begin, host_end), with buffers that hold only what those
+ * hosts need:
+ *   q, out  [(host_end-host_begin)*n, Hq, d]: the hosts' rows, in host order;
+ *   kv_k, kv_v [A + (host_end-host_begin)*n, Hkv, d]: the anchor's A rows
+ *           (the start of the sequence, which every host prepends to its
+ *           block), then the hosts' rows;
+ *   pass_k, pass_v [H*keep, Hkv, d]: all hosts' compressed blocks in host
+ *           order (rows [0, (host_end-1)*keep) are read);
+ *   lse [Hq, (host_end-host_begin)*n] (may be NULL).
+ * 0 <= host_begin < host_end <= n_hosts, else APB_ERR_INVALID_ARG. */
+apb_status apb_block_attention_hosts(const apb_config* cfg, int32_t host_begin, int32_t host_end,
+                                     const void* q, const void* kv_k, const void* kv_v,
+                                     const void* pass_k, const void* pass_v, void* out,
+                                     float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /* No counterpart in the paper: an allocation-free variant of
  * apb_score_compress, for callers that cannot hand this library any device

@@ -45,6 +45,9 @@ _lib.apb_build_passing.argtypes = [ctypes.POINTER(Config)] + [_P] * 6
 _lib.apb_build_passing.restype = ctypes.c_int
 _lib.apb_block_attention.argtypes = [ctypes.POINTER(Config)] + [_P] * 8 + [ctypes.c_size_t, _P]
 _lib.apb_block_attention.restype = ctypes.c_int
+_lib.apb_block_attention_hosts.argtypes = ([ctypes.POINTER(Config), ctypes.c_int32, ctypes.c_int32]
+                                           + [_P] * 8 + [ctypes.c_size_t, _P])
+_lib.apb_block_attention_hosts.restype = ctypes.c_int
 _lib.apb_score_compress_static.argtypes = [ctypes.POINTER(Config)] + [_P] * 9
 _lib.apb_score_compress_static.restype = ctypes.c_int
 _lib.apb_score_compress_static_max_floats.argtypes = []
@@ -183,12 +186,12 @@ def score_compress_static(c: Config, q, k, v, w1, b1, w2, b2, idx=None, stream=N
 
 
 def build_passing(c: Config, k, v, idx, pass_k=None, pass_v=None, stream=None):
-    """apb_build_passing: returns (pass_k, pass_v) [Hkv, H*keep, d] bf16."""
+    """apb_build_passing: returns (pass_k, pass_v) [H*keep, Hkv, d] bf16."""
     N, hq, hkv, d = _dims(c)
     _want(k, "k", torch.bfloat16, (N, hkv, d))
     _want(v, "v", torch.bfloat16, (N, hkv, d))
     _want(idx, "idx", torch.int32, (c.n_hosts, hkv, c.keep))
-    shape = (hkv, c.n_hosts * c.keep, d)
+    shape = (c.n_hosts * c.keep, hkv, d)
     if pass_k is None:
         pass_k = torch.empty(shape, dtype=torch.bfloat16, device=k.device)
     if pass_v is None:
@@ -212,7 +215,7 @@ def block_attention(c: Config, q, k, v, pass_k, pass_v, out=None, lse=None, want
     _want(v, "v", torch.bfloat16, (N, hkv, d))
     use_pass = c.keep > 0 and c.n_hosts > 1
     if use_pass:
-        shape = (hkv, c.n_hosts * c.keep, d)
+        shape = (c.n_hosts * c.keep, hkv, d)
         _want(pass_k, "pass_k", torch.bfloat16, shape)
         _want(pass_v, "pass_v", torch.bfloat16, shape)
     if out is None:
@@ -229,6 +232,39 @@ def block_attention(c: Config, q, k, v, pass_k, pass_v, out=None, lse=None, want
                                   _ptr(pass_v) if use_pass else None, _ptr(out), _ptr(lse),
                                   _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "apb_block_attention")
+    return out, lse
+
+
+def block_attention_hosts(c: Config, host_begin: int, host_end: int, q, kv_k, kv_v, pass_k,
+                          pass_v, out=None, lse=None, want_lse=False, workspace=None,
+                          stream=None):
+    """apb_block_attention_hosts: attention of hosts [host_begin, host_end)
+    on rank-local buffers (q/out: those hosts' rows; kv_k/kv_v: the anchor's
+    rows, then those hosts' rows).  Returns (out, lse or None)."""
+    _, hq, hkv, d = _dims(c)
+    rows = (host_end - host_begin) * c.block_len
+    _want(q, "q", torch.bfloat16, (rows, hq, d))
+    _want(kv_k, "kv_k", torch.bfloat16, (c.anchor_len + rows, hkv, d))
+    _want(kv_v, "kv_v", torch.bfloat16, (c.anchor_len + rows, hkv, d))
+    use_pass = c.keep > 0 and host_end > 1
+    if use_pass:
+        shape = (c.n_hosts * c.keep, hkv, d)
+        _want(pass_k, "pass_k", torch.bfloat16, shape)
+        _want(pass_v, "pass_v", torch.bfloat16, shape)
+    if out is None:
+        out = torch.empty((rows, hq, d), dtype=torch.bfloat16, device=q.device)
+    _want(out, "out", torch.bfloat16, (rows, hq, d))
+    if lse is None and want_lse:
+        lse = torch.empty((hq, rows), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (hq, rows))
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    st = _lib.apb_block_attention_hosts(ctypes.byref(c), host_begin, host_end, _ptr(q), _ptr(kv_k),
+                                        _ptr(kv_v), _ptr(pass_k) if use_pass else None,
+                                        _ptr(pass_v) if use_pass else None, _ptr(out), _ptr(lse),
+                                        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "apb_block_attention_hosts")
     return out, lse
 
 
@@ -257,7 +293,7 @@ class Prefill:
         self.c = c
         self.workspace = new_workspace(c, device)
         self.idx = torch.empty((c.n_hosts, hkv, c.keep), dtype=torch.int32, device=device)
-        shape = (hkv, c.n_hosts * c.keep, d)
+        shape = (c.n_hosts * c.keep, hkv, d)
         self.pass_k = torch.empty(shape, dtype=torch.bfloat16, device=device)
         self.pass_v = torch.empty(shape, dtype=torch.bfloat16, device=device)
         self.out = torch.empty((N, hq, d), dtype=torch.bfloat16, device=device)

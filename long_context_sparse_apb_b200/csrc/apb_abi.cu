@@ -157,35 +157,74 @@ apb_status apb_build_passing(const apb_config* cfg, const void* k, const void* v
   return APB_OK;
 }
 
-apb_status apb_block_attention(const apb_config* cfg, const void* q, const void* k,
-                               const void* v, const void* pass_k, const void* pass_v,
-                               void* out, float* lse, void* workspace, size_t ws_bytes,
-                               void* stream) {
+static apb_status attention_impl(const char* who, const apb_config* cfg, int hb, int he,
+                                 bool local, const void* q, const void* k, const void* v,
+                                 const void* pass_k, const void* pass_v, void* out, float* lse,
+                                 void* workspace, size_t ws_bytes, void* stream) {
   apb::Shape s;
   apb_status st = check_config(cfg, &s);
   if (st != APB_OK) return st;
+  if (hb < 0 || he > s.H || hb >= he)
+    return fail(APB_ERR_INVALID_ARG, "%s: host range [%d, %d) not inside [0, %d)", who, hb, he,
+                s.H);
   if (!q || !k || !v || !out || !workspace)
-    return fail(APB_ERR_INVALID_ARG, "apb_block_attention: NULL q/k/v/out/workspace");
-  bool need_pass = s.keep > 0 && s.H > 1;
+    return fail(APB_ERR_INVALID_ARG, "%s: NULL q/k/v/out/workspace", who);
+  // hosts h >= 1 read pass rows [0, h*keep)
+  const bool need_pass = s.keep > 0 && he > 1;
   if (need_pass && (!pass_k || !pass_v))
-    return fail(APB_ERR_INVALID_ARG, "apb_block_attention: NULL pass_k/pass_v with keep > 0");
+    return fail(APB_ERR_INVALID_ARG, "%s: NULL pass_k/pass_v with keep > 0", who);
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace) ||
       (need_pass && (!aligned16(pass_k) || !aligned16(pass_v))) || (lse && !aligned16(lse)))
-    return fail(APB_ERR_INVALID_ARG, "apb_block_attention: pointers must be 16-byte aligned");
+    return fail(APB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
   if (ws_bytes < apb::kStatusBytes)
-    return fail(APB_ERR_INVALID_ARG, "apb_block_attention: workspace %zu < %zu bytes", ws_bytes,
+    return fail(APB_ERR_INVALID_ARG, "%s: workspace %zu < %zu bytes", who, ws_bytes,
                 apb::kStatusBytes);
+  apb::HostRange r;
+  r.hb = hb;
+  r.he = he;
+  if (local) {
+    // rank-local buffers: Q/out hold hosts [hb, he); K/V hold the anchor rows
+    // [0, A) followed by those hosts' rows
+    r.q_row0 = 0;
+    r.k_row0 = s.A;
+    r.anchor_row0 = 0;
+    r.q_rows = (long long)(he - hb) * s.n;
+    r.k_rows = s.A + r.q_rows;
+  } else {
+    r.q_row0 = hb * s.n;
+    r.k_row0 = hb * s.n;
+    r.anchor_row0 = 0;
+    r.q_rows = s.N;
+    r.k_rows = s.N;
+  }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   auto* status = static_cast<apb::DeviceStatus*>(workspace);
   // clear the in-launch abort flag (the sticky bits stay until cleared)
   cudaError_t e = cudaMemsetAsync(&status->abort, 0, sizeof(uint32_t), cs);
   if (e != cudaSuccess) return cuda_fail(e, "clearing abort flag");
   const char* why = nullptr;
-  e = apb::launch_attention(s, q, k, v, need_pass ? pass_k : nullptr, need_pass ? pass_v : nullptr,
-                            out, lse, status, cs, &why);
+  e = apb::launch_attention(s, r, q, k, v, need_pass ? pass_k : nullptr,
+                            need_pass ? pass_v : nullptr, out, lse, status, cs, &why);
   if (why) return fail(APB_ERR_CUDA, "attention: %s", why);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
   return APB_OK;
+}
+
+apb_status apb_block_attention(const apb_config* cfg, const void* q, const void* k,
+                               const void* v, const void* pass_k, const void* pass_v,
+                               void* out, float* lse, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  const int H = cfg ? cfg->n_hosts : 1;
+  return attention_impl("apb_block_attention", cfg, 0, H, false, q, k, v, pass_k, pass_v, out, lse,
+                        workspace, ws_bytes, stream);
+}
+
+apb_status apb_block_attention_hosts(const apb_config* cfg, int32_t host_begin, int32_t host_end,
+                                     const void* q, const void* kv_k, const void* kv_v,
+                                     const void* pass_k, const void* pass_v, void* out,
+                                     float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return attention_impl("apb_block_attention_hosts", cfg, host_begin, host_end, true, q, kv_k,
+                        kv_v, pass_k, pass_v, out, lse, workspace, ws_bytes, stream);
 }
 
 apb_status apb_device_status(void* workspace, void* stream, int clear) {

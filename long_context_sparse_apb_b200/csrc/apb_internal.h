@@ -50,10 +50,18 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* idx, cudaStream_t st);
 cudaError_t launch_gather(const Shape& s, const void* k, const void* v, const int32_t* idx,
                           void* pass_k, void* pass_v, cudaStream_t st);
-// Returns cudaSuccess or an error; sets *encode_failed when a TMA descriptor
-// could not be built (reported as APB_ERR_CUDA with a message).
-cudaError_t launch_attention(const Shape& s, const void* q, const void* k, const void* v,
-                             const void* pass_k, const void* pass_v, void* out, float* lse,
-                             DeviceStatus* status, cudaStream_t st, const char** why);
+// Hosts [hb, he) of one attention launch and where their rows sit: row of
+// host hb's first token in the Q/out buffer (q_row0) and in the K/V buffer
+// (k_row0), row of the anchor's first token in K/V, and the buffers' rows.
+struct HostRange {
+  int hb, he, q_row0, k_row0, anchor_row0;
+  long long q_rows, k_rows;
+};
+
+// Returns cudaSuccess or an error; sets *why when a TMA descriptor could not
+// be built (reported as APB_ERR_CUDA with a message).
+cudaError_t launch_attention(const Shape& s, const HostRange& r, const void* q, const void* k,
+                             const void* v, const void* pass_k, const void* pass_v, void* out,
+                             float* lse, DeviceStatus* status, cudaStream_t st, const char** why);
 
 }  // namespace apb

@@ -88,7 +88,10 @@ constexpr int kSmemBytes = Layout<128>::kBytes + 1024;
 
 struct Params {
   int H, n, A, keep, Hq, Hkv, G, n_ctas_per_host;
-  long long N;
+  // hosts [hb, he) of this launch; rows, in the Q/out and K/V buffers, of the
+  // first token of host hb, and, in K/V, of the anchor's first token
+  int hb, he, q_row0, k_row0, anchor_row0;
+  long long N;   // rows of the Q/out buffer (the lse row stride)
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
@@ -98,15 +101,15 @@ struct Params {
 template <int D>
 __device__ __forceinline__ void load_kv_tile(const CUtensorMap* m_kv, const CUtensorMap* m_pass,
                                              uint8_t* dst, uint64_t* bar, int j, int na, int np,
-                                             int g, int local_row0) {
+                                             int g, int local_row0, int anchor_row0) {
   if (j < na) {
 #pragma unroll
     for (int kb = 0; kb < D / 64; ++kb)
-      ptx::tma_load_3d(dst + kb * (kRows * 128), m_kv, bar, kb * 64, g, j * kRows);
+      ptx::tma_load_3d(dst + kb * (kRows * 128), m_kv, bar, kb * 64, g, anchor_row0 + j * kRows);
   } else if (j < na + np) {
 #pragma unroll
     for (int kb = 0; kb < D / 64; ++kb)
-      ptx::tma_load_3d(dst + kb * (kRows * 128), m_pass, bar, kb * 64, (j - na) * kRows, g);
+      ptx::tma_load_3d(dst + kb * (kRows * 128), m_pass, bar, kb * 64, g, (j - na) * kRows);
   } else {
 #pragma unroll
     for (int kb = 0; kb < D / 64; ++kb)
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // heavy units first: the last query tiles of the last hosts
   const int u = p.n_ctas_per_host - 1 - (int)blockIdx.x;
   const int head = (int)blockIdx.y;
-  const int h = p.H - 1 - (int)blockIdx.z;
+  const int h = p.he - 1 - (int)blockIdx.z;
   const int g = head / p.G;
   const int qA0 = 2 * u * kRows;                 // first local row of tile A
   const int na = (h >= 1 && p.A > 0) ? (p.A + kRows - 1) / kRows : 0;
@@ -145,7 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int TA = na + np + 2 * u + 1;            // KV tiles of query tile A
   const int TB = (qA0 + kRows < p.n) ? TA + 1 : 0;   // of tile B (0: beyond the block)
   const int Tmax = TB > 0 ? TB : TA;
-  const int local_row0 = h * p.n;                // first K row of this host's block
+  const int local_row0 = p.k_row0 + (h - p.hb) * p.n;   // K/V row of this host's token 0
+  const int q_row0 = p.q_row0 + (h - p.hb) * p.n;       // Q/out row of this host's token 0
 
   const volatile uint32_t* gabort = &p.status->abort;
 
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb)
           ptx::tma_load_3d(sQ + i * L::kTile + kb * (kRows * 128), &mQ, &bars[Q_FULL], kb * 64,
-                           head, local_row0 + qA0 + i * kRows);
+                           head, q_row0 + qA0 + i * kRows);
       }
       for (int j = 0; j < Tmax; ++j) {
         const int ks = j % kKStages, vs = j % kVStages;
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::mbar_arrive_expect_tx(&bars[K_FULL + ks], L::kTile);
         load_kv_tile<D>(&mK, &mPK, sK0 + ks * L::kTile, &bars[K_FULL + ks], j, na, np, g,
-                        local_row0);
+                        local_row0, p.anchor_row0);
         lastK[ks] = (int)kpar;
         if (!ptx::mbar_wait_bounded(&bars[V_EMPTY + vs], vpar ^ 1, gabort, kWaitLimitNs)) {
           record_failure(p.status, 42 + vs, j);
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::mbar_arrive_expect_tx(&bars[V_FULL + vs], L::kTile);
         load_kv_tile<D>(&mV, &mPV, sV0 + vs * L::kTile, &bars[V_FULL + vs], j, na, np, g,
-                        local_row0);
+                        local_row0, p.anchor_row0);
         lastV[vs] = (int)vpar;
       }
       // drain: every load issued must have landed before the CTA exits
@@ -425,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         const float inv = 1.0f / l;
         const bool valid = q0 + row < p.n;
-        const long long tok = (long long)local_row0 + q0 + row;
+        const long long tok = (long long)q_row0 + q0 + row;
         __nv_bfloat16* orow = p.out + (tok * p.Hq + head) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -460,23 +464,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------- host side
 
 template <int D>
-cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v,
-                     const void* pass_k, const void* pass_v, void* out, float* lse,
+cudaError_t launch_d(const Shape& s, const HostRange& r, const void* q, const void* k,
+                     const void* v, const void* pass_k, const void* pass_v, void* out, float* lse,
                      DeviceStatus* status, cudaStream_t st, const char** why) {
   CUtensorMap mQ, mK, mV, mPK, mPV;
-  const uint64_t N = (uint64_t)s.N;
-  bool ok = encode_bf16_3d(&mQ, q, D, s.Hq, N, (uint64_t)D * 2, (uint64_t)s.Hq * D * 2, 64, 1,
+  const uint64_t NQ = (uint64_t)r.q_rows, NK = (uint64_t)r.k_rows;
+  bool ok = encode_bf16_3d(&mQ, q, D, s.Hq, NQ, (uint64_t)D * 2, (uint64_t)s.Hq * D * 2, 64, 1,
                            kRows) &&
-            encode_bf16_3d(&mK, k, D, s.Hkv, N, (uint64_t)D * 2, (uint64_t)s.Hkv * D * 2, 64, 1,
+            encode_bf16_3d(&mK, k, D, s.Hkv, NK, (uint64_t)D * 2, (uint64_t)s.Hkv * D * 2, 64, 1,
                            kRows) &&
-            encode_bf16_3d(&mV, v, D, s.Hkv, N, (uint64_t)D * 2, (uint64_t)s.Hkv * D * 2, 64, 1,
+            encode_bf16_3d(&mV, v, D, s.Hkv, NK, (uint64_t)D * 2, (uint64_t)s.Hkv * D * 2, 64, 1,
                            kRows);
   if (ok && pass_k) {
+    // token-major [H*keep, Hkv, d], read like K
     const uint64_t rows = (uint64_t)s.H * s.keep;
-    ok = encode_bf16_3d(&mPK, pass_k, D, rows, s.Hkv, (uint64_t)D * 2, rows * D * 2, 64, kRows,
-                        1) &&
-         encode_bf16_3d(&mPV, pass_v, D, rows, s.Hkv, (uint64_t)D * 2, rows * D * 2, 64, kRows,
-                        1);
+    ok = encode_bf16_3d(&mPK, pass_k, D, s.Hkv, rows, (uint64_t)D * 2, (uint64_t)s.Hkv * D * 2,
+                        64, 1, kRows) &&
+         encode_bf16_3d(&mPV, pass_v, D, s.Hkv, rows, (uint64_t)D * 2, (uint64_t)s.Hkv * D * 2,
+                        64, 1, kRows);
   } else {
     mPK = mK;   // no passing block: never loaded
     mPV = mV;
@@ -494,7 +499,12 @@ cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v
   p.Hkv = s.Hkv;
   p.G = s.Hq / s.Hkv;
   p.n_ctas_per_host = ((s.n + kRows - 1) / kRows + 1) / 2;
-  p.N = s.N;
+  p.hb = r.hb;
+  p.he = r.he;
+  p.q_row0 = r.q_row0;
+  p.k_row0 = r.k_row0;
+  p.anchor_row0 = r.anchor_row0;
+  p.N = r.q_rows;
   p.scale_log2 = s.scale * kLog2e;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
@@ -502,18 +512,18 @@ cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v
   cudaError_t e = cudaFuncSetAttribute(apb_attention_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_ctas_per_host, s.Hq, s.H);
+  dim3 grid(p.n_ctas_per_host, s.Hq, r.he - r.hb);
   apb_attention_kernel<D><<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, mPK, mPV, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attention(const Shape& s, const void* q, const void* k, const void* v,
-                             const void* pass_k, const void* pass_v, void* out, float* lse,
-                             DeviceStatus* status, cudaStream_t st, const char** why) {
-  if (s.d == 128) return launch_d<128>(s, q, k, v, pass_k, pass_v, out, lse, status, st, why);
-  return launch_d<64>(s, q, k, v, pass_k, pass_v, out, lse, status, st, why);
+cudaError_t launch_attention(const Shape& s, const HostRange& r, const void* q, const void* k,
+                             const void* v, const void* pass_k, const void* pass_v, void* out,
+                             float* lse, DeviceStatus* status, cudaStream_t st, const char** why) {
+  if (s.d == 128) return launch_d<128>(s, r, q, k, v, pass_k, pass_v, out, lse, status, st, why);
+  return launch_d<64>(s, r, q, k, v, pass_k, pass_v, out, lse, status, st, why);
 }
 
 }  // namespace apb

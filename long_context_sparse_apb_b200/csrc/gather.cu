@@ -1,7 +1,10 @@
 // Passing-block construction: the on-GPU stand-in for the all-gather of
 // compressed blocks ("APB 的主要功能", communication).  With H virtual hosts
 // on one GPU the all-gather is a gather in HBM:
-//     pass[g, h*keep + r, :] = src[idx[h, g, r], g, :]      (K and V)
+//     pass[h*keep + r, g, :] = src[idx[h, g, r], g, :]      (K and V)
+// The passing layout is token-major like K and V, so host h's passing block
+// is the prefix of h*keep rows and the blocks of a range of hosts are one
+// contiguous chunk (what a multi-GPU all-gather exchanges).
 // Each output row is d bf16 = 128 or 256 bytes; consecutive threads copy
 // consecutive 16-byte chunks of a row, so reads of a source row and writes of
 // the destination rows are both fully coalesced.
@@ -25,7 +28,7 @@ __global__ void __launch_bounds__(256) gather_passing_kernel(
     const int g = (int)(hg % Hkv);
     const int h = (int)(hg / Hkv);
     const long long t = __ldg(idx + row);
-    const long long dst = ((long long)g * H * keep + (long long)h * keep + r) * chunks_per_row + c;
+    const long long dst = (((long long)h * keep + r) * Hkv + g) * chunks_per_row + c;
     uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
     if (t >= 0 && t < N) {
       const long long src = (t * Hkv + g) * chunks_per_row + c;

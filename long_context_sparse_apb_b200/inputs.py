@@ -142,6 +142,39 @@ def generate_weights(cfg: APBConfig) -> Dict[str, torch.Tensor]:
             "w2": w2.contiguous(), "b2": b2.contiguous()}
 
 
+def _q_block(cfg: APBConfig, h: int) -> torch.Tensor:
+    """Host h's post-RoPE fp32 Q block [n, Hq, d]."""
+    n, d = cfg.block_len, cfg.head_dim
+    x = torch.randn((n, cfg.n_q_heads, d), generator=_gen(mix(cfg.seed, _TID_Q, h)))
+    if cfg.rope_theta is not None:
+        _rope_(x, h * n, cfg.rope_theta)
+    return x
+
+
+def _qseg_mean(cfg: APBConfig, q0: torch.Tensor) -> torch.Tensor:
+    """[Hkv, d] mean of post-RoPE fp32 Q over the query segment and the group."""
+    hkv, G, d = cfg.n_kv_heads, cfg.group, cfg.head_dim
+    if cfg.query_len == 0:
+        return torch.zeros(hkv, d)
+    return q0[: cfg.query_len].reshape(cfg.query_len, hkv, G, d).mean(dim=(0, 2))
+
+
+def _kv_block(cfg: APBConfig, h: int, qseg_mean: torch.Tensor, which: int) -> torch.Tensor:
+    """Host h's K (which = K id, needles planted) or V block, fp32."""
+    n, d, hkv = cfg.block_len, cfg.head_dim, cfg.n_kv_heads
+    x = torch.randn((n, hkv, d), generator=_gen(mix(cfg.seed, which, h)))
+    if which == _TID_K:
+        if cfg.rope_theta is not None:
+            _rope_(x, h * n, cfg.rope_theta)
+        pos = needle_positions(cfg, h)
+        if pos.numel():
+            u = qseg_mean / qseg_mean.norm(dim=-1, keepdim=True).clamp_min(1e-30)
+            x[pos - h * n] = (3.0 * math.sqrt(d) * u)[None, :, :]
+    elif cfg.v_std != 1.0:
+        x *= cfg.v_std
+    return x
+
+
 def generate(cfg: APBConfig) -> Dict[str, torch.Tensor]:
     """All inputs of one workload as CPU tensors.
 
@@ -149,39 +182,44 @@ def generate(cfg: APBConfig) -> Dict[str, torch.Tensor]:
     w1/b1/w2/b2 (fp32) and ``needles`` (int64 global positions).
     """
     H, n, d = cfg.n_hosts, cfg.block_len, cfg.head_dim
-    hq, hkv, G = cfg.n_q_heads, cfg.n_kv_heads, cfg.group
+    hq, hkv = cfg.n_q_heads, cfg.n_kv_heads
     N = H * n
     q = torch.empty((N, hq, d), dtype=torch.bfloat16)
     k = torch.empty((N, hkv, d), dtype=torch.bfloat16)
     v = torch.empty((N, hkv, d), dtype=torch.bfloat16)
-
-    qseg_mean = None  # [Hkv, d] mean of post-RoPE fp32 Q over the query segment
+    qseg_mean = None
     for h in range(H):
-        x = torch.randn((n, hq, d), generator=_gen(mix(cfg.seed, _TID_Q, h)))
-        if cfg.rope_theta is not None:
-            _rope_(x, h * n, cfg.rope_theta)
+        x = _q_block(cfg, h)
         if h == 0:
-            seg = x[: cfg.query_len].reshape(cfg.query_len, hkv, G, d)
-            qseg_mean = seg.mean(dim=(0, 2)) if cfg.query_len > 0 else torch.zeros(hkv, d)
+            qseg_mean = _qseg_mean(cfg, x)
         q[h * n:(h + 1) * n] = x.to(torch.bfloat16)
     for h in range(H):
-        x = torch.randn((n, hkv, d), generator=_gen(mix(cfg.seed, _TID_K, h)))
-        if cfg.rope_theta is not None:
-            _rope_(x, h * n, cfg.rope_theta)
-        pos = needle_positions(cfg, h)
-        if pos.numel():
-            u = qseg_mean / qseg_mean.norm(dim=-1, keepdim=True).clamp_min(1e-30)
-            x[pos - h * n] = (3.0 * math.sqrt(d) * u)[None, :, :]
-        k[h * n:(h + 1) * n] = x.to(torch.bfloat16)
+        k[h * n:(h + 1) * n] = _kv_block(cfg, h, qseg_mean, _TID_K).to(torch.bfloat16)
     for h in range(H):
-        x = torch.randn((n, hkv, d), generator=_gen(mix(cfg.seed, _TID_V, h)))
-        if cfg.v_std != 1.0:
-            x *= cfg.v_std
-        v[h * n:(h + 1) * n] = x.to(torch.bfloat16)
+        v[h * n:(h + 1) * n] = _kv_block(cfg, h, qseg_mean, _TID_V).to(torch.bfloat16)
 
     out = {"q": q, "k": k, "v": v}
     out.update(generate_weights(cfg))
     out["needles"] = torch.cat([needle_positions(cfg, h) for h in range(H)])
+    return out
+
+
+def generate_local(cfg: APBConfig, host_begin: int, host_end: int) -> Dict[str, torch.Tensor]:
+    """What one GPU of a host-sharded prefill holds: q of hosts
+    [host_begin, host_end) and k/v with the anchor's rows [0, A) first, then
+    those hosts' rows (each host prepends the anchor to its block).  Values
+    equal the matching rows of generate(cfg)."""
+    n, A = cfg.block_len, cfg.anchor_len
+    q0 = _q_block(cfg, 0)
+    qseg_mean = _qseg_mean(cfg, q0)
+    hosts = range(host_begin, host_end)
+    q = torch.cat([(q0 if h == 0 else _q_block(cfg, h)).to(torch.bfloat16) for h in hosts])
+    out = {"q": q}
+    for name, tid in (("k", _TID_K), ("v", _TID_V)):
+        anchor = _kv_block(cfg, 0, qseg_mean, tid)[:A].to(torch.bfloat16)
+        blocks = [_kv_block(cfg, h, qseg_mean, tid).to(torch.bfloat16) for h in hosts]
+        out[name] = torch.cat([anchor] + blocks)
+    out.update(generate_weights(cfg))
     return out
 
 

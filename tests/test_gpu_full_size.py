@@ -48,13 +48,13 @@ def test_full_size_workload(apb, name):
     check_topk(idx, s_ref, cfg)
     k16, v16 = x["k"].view(torch.int16).numpy(), x["v"].view(torch.int16).numpy()
     rk, rv = oracle.passing_blocks(k16, v16, idx.astype(np.int64))
-    pk16 = run.pass_k.view(torch.int16).cpu().numpy()
-    pv16 = run.pass_v.view(torch.int16).cpu().numpy()
+    pk16 = run.pass_k.view(torch.int16).permute(1, 0, 2).cpu().numpy()
+    pv16 = run.pass_v.view(torch.int16).permute(1, 0, 2).cpu().numpy()
     assert np.array_equal(pk16, rk) and np.array_equal(pv16, rv)
 
     k, v = f32np(x["k"]), f32np(x["v"])
-    pkn = f32np(run.pass_k.cpu())
-    pvn = f32np(run.pass_v.cpu())
+    pkn = f32np(run.pass_k.permute(1, 0, 2).cpu())
+    pvn = f32np(run.pass_v.permute(1, 0, 2).cpu())
     n, G = cfg.block_len, cfg.group
     nrows = cfg.sample_rows_per_host or 512
     for h in range(cfg.n_hosts):

@@ -54,8 +54,9 @@ def _check_passing_exact(x, idx_np, pk, pv):
     k16 = x["k"].view(torch.int16).numpy()
     v16 = x["v"].view(torch.int16).numpy()
     rk, rv = oracle.passing_blocks(k16, v16, idx_np.astype(np.int64))
-    assert np.array_equal(pk.view(torch.int16).cpu().numpy(), rk)
-    assert np.array_equal(pv.view(torch.int16).cpu().numpy(), rv)
+    # device layout [H*keep, Hkv, d]; the oracle's [Hkv, H*keep, d]
+    assert np.array_equal(pk.view(torch.int16).permute(1, 0, 2).cpu().numpy(), rk)
+    assert np.array_equal(pv.view(torch.int16).permute(1, 0, 2).cpu().numpy(), rv)
 
 
 def _full_parity(apb, cfg, x=None):
@@ -69,7 +70,7 @@ def _full_parity(apb, cfg, x=None):
         check_topk(idx_np, s_ref, cfg)
     _check_passing_exact(x, idx_np, pk, pv)
     k, v = f32np(x["k"]), f32np(x["v"])
-    pkn, pvn = f32np(pk.cpu()), f32np(pv.cpu())
+    pkn, pvn = f32np(pk.permute(1, 0, 2).cpu()), f32np(pv.permute(1, 0, 2).cpu())
     n = cfg.block_len
     o_all = out.float().cpu().numpy()
     lse_all = lse.cpu().numpy()

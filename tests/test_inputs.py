@@ -40,3 +40,16 @@ def test_sample_rows_hold_edges():
     assert torch.all(r[1:] > r[:-1])
     for must in (0, cfg.block_len - 1, cfg.anchor_len - 1, 127, 128):
         assert must in r.tolist()
+
+
+def test_generate_local_matches_full_sequence():
+    cfg = inputs.TINY
+    x = inputs.generate(cfg)
+    n, A = cfg.block_len, cfg.anchor_len
+    for hb, he in ((0, 2), (2, 4), (1, 4), (3, 4)):
+        loc = inputs.generate_local(cfg, hb, he)
+        assert torch.equal(loc["q"], x["q"][hb * n:he * n])
+        for t in ("k", "v"):
+            assert torch.equal(loc[t][:A], x[t][:A])
+            assert torch.equal(loc[t][A:], x[t][hb * n:he * n])
+        assert torch.equal(loc["w1"], x["w1"])
