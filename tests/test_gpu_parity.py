@@ -180,3 +180,33 @@ def test_query_aware_scores_and_selection(apb, cfg):
     idx2, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"],
                                  xd["b2"], workspace=ws)
     assert idx2.shape == idx.shape
+
+
+def _random_shapes(count, seed=2026):
+    rng = np.random.default_rng(seed)
+    shapes = [
+        # degenerate cases first: one-token blocks, anchor = whole block, keep = n = 1
+        (3, 1, 1, 1, 1, 2, 1, 64),
+        (2, 1, 0, 0, 0, 4, 4, 128),
+        (1, 5, 5, 2, 5, 8, 1, 128),          # one host, G = 8
+    ]
+    while len(shapes) < count:
+        H = int(rng.integers(1, 6))
+        n = int(rng.integers(2, 700))
+        A = int(rng.integers(0, n + 1))
+        ql = int(rng.integers(0, A + 1))
+        keep = int(rng.choice([0, 1, int(rng.integers(1, n + 1)), n]))
+        hkv = int(rng.choice([1, 2, 4]))
+        G = int(rng.choice([1, 2, 4, 5, 8]))
+        d = int(rng.choice([64, 128]))
+        shapes.append((H, n, A, ql, keep, hkv * G, hkv, d))
+    return shapes
+
+
+@pytest.mark.parametrize("shape", _random_shapes(14), ids=lambda s: "x".join(map(str, s)))
+def test_random_shapes_every_row(apb, shape):
+    H, n, A, ql, keep, hq, hkv, d = shape
+    cfg = inputs.APBConfig("rand", n_hosts=H, block_len=n, anchor_len=A, query_len=ql, keep=keep,
+                           n_q_heads=hq, n_kv_heads=hkv, head_dim=d, seed=31 + H + n + keep,
+                           rope_theta=1e4 if d == 128 else None, needles_per_host=1)
+    _full_parity(apb, cfg)
