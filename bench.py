@@ -265,26 +265,29 @@ def run_gpu(args, cfg):
 
     n_ev = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_ev)]
+    # the timed step: the whole path in one C call (apb_prefill)
+    pws = torch.zeros(apb.prefill_workspace_bytes(c), dtype=torch.uint8, device=dev)
+    pout = torch.empty_like(run.out)
 
-    def step(e=None):
-        if e is not None:
-            e[0].record(stream)
+    def step():
+        apb.prefill(c, xd["q"], xd["k"], xd["v"], *w, out=pout, workspace=pws, stream=stream)
+
+    # the same path as three calls, for the per-stage breakdown
+    def staged(e):
+        e[0].record(stream)
         apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, idx=run.idx,
                            workspace=run.workspace, stream=stream)
-        if e is not None:
-            e[1].record(stream)
+        e[1].record(stream)
         apb.build_passing(c, xd["k"], xd["v"], run.idx, run.pass_k, run.pass_v, stream=stream)
-        if e is not None:
-            e[2].record(stream)
+        e[2].record(stream)
         apb.block_attention(c, xd["q"], xd["k"], xd["v"], run.pass_k, run.pass_v, out=run.out,
                             workspace=run.workspace, stream=stream)
-        if e is not None:
-            e[3].record(stream)
+        e[3].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    if apb.device_status(run.workspace) != apb.APB_OK:
+    if apb.device_status(pws) != apb.APB_OK:
         raise RuntimeError("device status not OK after warm-up")
 
     clocks = ClockSampler(local)
@@ -295,15 +298,18 @@ def run_gpu(args, cfg):
     torch.cuda.synchronize(dev)
     t_start.record(stream)
     for i in range(args.steps):
-        step(ev[i])
+        step()
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     clk = clocks.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
-    status = apb.device_status(run.workspace)
+    status = apb.device_status(pws)
     if status != apb.APB_OK:
         raise RuntimeError(f"device status {apb.status_string(status)} after timed steps")
+    for i in range(n_ev):
+        staged(ev[i])
+    torch.cuda.synchronize(dev)
 
     score_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     gather_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
@@ -319,7 +325,7 @@ def run_gpu(args, cfg):
     hout = [torch.empty(run.out.shape, dtype=run.out.dtype).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in hx.values())
     d2h = hout[0].numel() * hout[0].element_size()
-    del run, xd
+    del run, xd, pws, pout
     torch.cuda.empty_cache()
     pipe = apb.PrefillPipeline(c, device=dev, depth=2)
     for i in range(max(2, args.warmup)):
@@ -396,10 +402,10 @@ def run_gpu(args, cfg):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms": e2e_ms,
                 "host_wall_ms": wall_ms,
-                "how": "PrefillPipeline: pinned H2D copies, the three calls and the D2H copy of "
+                "how": "PrefillPipeline: pinned H2D copies, one apb_prefill call and the D2H copy of "
                        "the output on three streams, two slots, copies of one step overlapping "
                        "another step's compute"},
-        "gpu_launches": args.steps * (5 if cfg.keep > 0 else 3),
+        "gpu_launches": args.steps * (5 if cfg.keep > 0 and cfg.n_hosts > 1 else 1),
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
@@ -533,6 +539,59 @@ def run_sharded(args, cfg):
         dist.destroy_process_group()
 
 
+def run_heads(args, cfg):
+    """One sequence prefilled by N GPUs, kv heads split evenly: each rank runs
+    the whole path on its kv heads and their q heads; no collective.  Strong
+    scaling: value = tokens of the one sequence / max-over-ranks step time."""
+    from long_context_sparse_apb_b200 import _lib as apb
+    from long_context_sparse_apb_b200.sharded import head_slice, kv_head_range
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    gb, ge = kv_head_range(cfg.n_kv_heads, rank, world)
+    G = cfg.group
+    loc = {k: v.to(dev) for k, v in
+           head_slice(inputs.generate(cfg), cfg.n_q_heads, cfg.n_kv_heads, gb, ge).items()}
+    c = apb.make_config(cfg, n_q_heads=(ge - gb) * G, n_kv_heads=ge - gb)
+    run = apb.Prefill(c, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    args_w = (loc["w1"], loc["b1"], loc["w2"], loc["b2"])
+    for _ in range(args.warmup):
+        run(loc["q"], loc["k"], loc["v"], *args_w, stream=stream)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        run(loc["q"], loc["k"], loc["v"], *args_w, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    if apb.device_status(run.workspace) != apb.APB_OK:
+        raise RuntimeError("device status not OK after timed steps")
+    max_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    if rank == 0:
+        cdict = config_dict(cfg, world)
+        cdict["parallelism"] = (f"kv-head-sharded: {world} GPU(s) x {ge - gb} kv head(s), "
+                                f"no collective")
+        line = {"metric": METRIC, "value": cfg.seq_len / (max_ms / 1e3 / args.steps),
+                "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": cdict, "e2e": None,
+                "e2e_note": "host-buffer end-to-end is measured in the default mode",
+                "gpu_launches": args.steps * (5 if cfg.keep else 3), "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def apb_kernel_rev() -> str:
     """Hash of the attention kernel source: ncu traffic counters only apply to
     the revision they were taken on."""
@@ -547,10 +606,12 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded"],
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded", "heads"],
                     help="replicas: one independent sequence per GPU (weak scaling); "
                          "sharded: one sequence with its hosts split over the GPUs and an "
-                         "NCCL all-gather of the compressed blocks (strong scaling)")
+                         "NCCL all-gather of the compressed blocks (strong scaling); "
+                         "heads: one sequence with its kv heads split over the GPUs, no "
+                         "collective (strong scaling)")
     ap.add_argument("--workload", default="llama8b_128k", choices=sorted(inputs.CONFIGS))
     ap.add_argument("--oracle-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -562,6 +623,8 @@ def main():
         run_reference(args, cfg)
     elif args.mode == "sharded":
         run_sharded(args, cfg)
+    elif args.mode == "heads":
+        run_heads(args, cfg)
     else:
         run_gpu(args, cfg)
 

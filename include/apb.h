@@ -172,6 +172,19 @@ apb_status apb_block_attention_hosts(const apb_config* cfg, int32_t host_begin, 
                                      const void* pass_k, const void* pass_v, void* out,
                                      float* lse, void* workspace, size_t ws_bytes, void* stream);
 
+/* The whole path in one call: steps 1-3 on one GPU for all hosts, writing
+ * out [N, Hq, d] (and lse [Hq, N] when not NULL).  The last host's
+ * compressed block is not computed: no host follows it, so no passing block
+ * contains it (main features: each passing block holds the preceding hosts'
+ * blocks); out and lse equal those of apb_score_compress + apb_build_passing
+ * + apb_block_attention.  workspace: apb_prefill_workspace_bytes(cfg) bytes,
+ * zero-filled before first use; it holds the scores, indices and passing
+ * blocks between the steps. */
+size_t apb_prefill_workspace_bytes(const apb_config* cfg);
+apb_status apb_prefill(const apb_config* cfg, const void* q, const void* k, const void* v,
+                       const float* w1, const float* b1, const float* w2, const float* b2,
+                       void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
 /* No counterpart in the paper: an allocation-free variant of
  * apb_score_compress, for callers that cannot hand this library any device
  * memory besides the tensors themselves (a host framework whose allocator

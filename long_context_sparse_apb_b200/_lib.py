@@ -41,6 +41,10 @@ _lib.apb_score_compress.argtypes = [ctypes.POINTER(Config)] + [_P] * 10 + [ctype
 _lib.apb_score_compress.restype = ctypes.c_int
 _lib.apb_score_compress_query_aware.argtypes = _lib.apb_score_compress.argtypes
 _lib.apb_score_compress_query_aware.restype = ctypes.c_int
+_lib.apb_prefill_workspace_bytes.argtypes = [ctypes.POINTER(Config)]
+_lib.apb_prefill_workspace_bytes.restype = ctypes.c_size_t
+_lib.apb_prefill.argtypes = [ctypes.POINTER(Config)] + [_P] * 10 + [ctypes.c_size_t, _P]
+_lib.apb_prefill.restype = ctypes.c_int
 _lib.apb_build_passing.argtypes = [ctypes.POINTER(Config)] + [_P] * 6
 _lib.apb_build_passing.restype = ctypes.c_int
 _lib.apb_block_attention.argtypes = [ctypes.POINTER(Config)] + [_P] * 8 + [ctypes.c_size_t, _P]
@@ -268,6 +272,37 @@ def block_attention_hosts(c: Config, host_begin: int, host_end: int, q, kv_k, kv
     return out, lse
 
 
+def prefill_workspace_bytes(c: Config) -> int:
+    return int(_lib.apb_prefill_workspace_bytes(ctypes.byref(c)))
+
+
+def prefill(c: Config, q, k, v, w1, b1, w2, b2, out=None, lse=None, want_lse=False,
+            workspace=None, stream=None):
+    """apb_prefill: the whole path in one call.  Returns (out, lse or None)."""
+    N, hq, hkv, d = _dims(c)
+    _want(q, "q", torch.bfloat16, (N, hq, d))
+    _want(k, "k", torch.bfloat16, (N, hkv, d))
+    _want(v, "v", torch.bfloat16, (N, hkv, d))
+    _want(w1, "w1", torch.float32, (hkv, c.mlp_hidden, 3 * d))
+    _want(b1, "b1", torch.float32, (hkv, c.mlp_hidden))
+    _want(w2, "w2", torch.float32, (hkv, c.mlp_hidden))
+    _want(b2, "b2", torch.float32, (hkv,))
+    if out is None:
+        out = torch.empty((N, hq, d), dtype=torch.bfloat16, device=q.device)
+    _want(out, "out", torch.bfloat16, (N, hq, d))
+    if lse is None and want_lse:
+        lse = torch.empty((hq, N), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (hq, N))
+    if workspace is None:
+        workspace = torch.zeros(prefill_workspace_bytes(c), dtype=torch.uint8, device=q.device)
+    st = _lib.apb_prefill(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1),
+                          _ptr(w2), _ptr(b2), _ptr(out), _ptr(lse), _ptr(workspace),
+                          workspace.numel(), _stream(stream))
+    _check(st, "apb_prefill")
+    return out, lse
+
+
 def device_status(workspace, stream=None, clear=False) -> int:
     """apb_device_status: synchronises the stream, returns the status code."""
     return int(_lib.apb_device_status(_ptr(workspace), _stream(stream), 1 if clear else 0))
@@ -311,8 +346,8 @@ class PrefillPipeline:
     """Prefills of successive sequences from pinned host memory with the
     transfers of one step overlapped with the compute of another.
 
-    Each of `depth` slots owns device copies of the inputs and a Prefill
-    (workspace, indices, passing block, output).  submit() queues, on three
+    Each of `depth` slots owns device copies of the inputs, an apb_prefill
+    workspace and an output buffer; the compute is one apb_prefill call.  submit() queues, on three
     streams ordered by events, the host->device copy of the step's inputs,
     the three calls of the path, and the device->host copy of the output into
     the caller's pinned buffer.  A slot's inputs are overwritten only after its
@@ -337,7 +372,10 @@ class PrefillPipeline:
                  "w2": torch.empty((hkv, c.mlp_hidden), dtype=torch.float32, device=dev),
                  "b2": torch.empty((hkv,), dtype=torch.float32, device=dev)}
             ev = {k: torch.cuda.Event() for k in ("in", "comp", "out")}
-            self.slots.append({"x": x, "run": Prefill(c, device=dev), "ev": ev, "used": False})
+            self.slots.append({"x": x, "ev": ev, "used": False,
+                               "ws": torch.zeros(prefill_workspace_bytes(c), dtype=torch.uint8,
+                                                 device=dev),
+                               "out": torch.empty((N, hq, d), dtype=torch.bfloat16, device=dev)})
         self.i = 0
 
     def submit(self, host: dict, host_out: torch.Tensor) -> None:
@@ -357,12 +395,12 @@ class PrefillPipeline:
             if slot["used"]:
                 self.comp.wait_event(ev["out"])          # previous output copied back
             x = slot["x"]
-            slot["run"](x["q"], x["k"], x["v"], x["w1"], x["b1"], x["w2"], x["b2"],
-                        stream=self.comp)
+            prefill(self.c, x["q"], x["k"], x["v"], x["w1"], x["b1"], x["w2"], x["b2"],
+                    out=slot["out"], workspace=slot["ws"], stream=self.comp)
             ev["comp"].record(self.comp)
         with torch.cuda.stream(self.d2h):
             self.d2h.wait_event(ev["comp"])
-            host_out.copy_(slot["run"].out, non_blocking=True)
+            host_out.copy_(slot["out"], non_blocking=True)
             ev["out"].record(self.d2h)
         slot["used"] = True
 

@@ -227,6 +227,80 @@ apb_status apb_block_attention_hosts(const apb_config* cfg, int32_t host_begin, 
                         kv_v, pass_k, pass_v, out, lse, workspace, ws_bytes, stream);
 }
 
+// ---------------------------------------------------------------- one call
+
+// Workspace of apb_prefill: status block, W1 split, query-aware bias slot,
+// then scores of hosts 0..H-2, their indices, and the passing K and V blocks
+// (H*keep rows each; the last host's rows are never written or read).
+struct PrefillLayout {
+  size_t wsplit, scores, idx, pass_k, pass_v, total;
+};
+
+static PrefillLayout prefill_layout(const apb::Shape& s) {
+  PrefillLayout L;
+  const size_t h1 = s.H > 1 ? (size_t)(s.H - 1) : 0;
+  const size_t pass = round256((size_t)s.H * s.keep * s.Hkv * s.d * 2);
+  L.wsplit = apb::kStatusBytes;
+  L.scores = L.wsplit + round256(apb::weight_split_bytes(s)) + round256(apb::query_bias_bytes(s));
+  L.idx = L.scores + round256(h1 * s.n * s.Hkv * sizeof(float));
+  L.pass_k = L.idx + round256(h1 * s.Hkv * s.keep * sizeof(int32_t));
+  L.pass_v = L.pass_k + pass;
+  L.total = L.pass_v + pass;
+  return L;
+}
+
+size_t apb_prefill_workspace_bytes(const apb_config* cfg) {
+  apb::Shape s;
+  if (check_config(cfg, &s) != APB_OK) return 0;
+  return prefill_layout(s).total;
+}
+
+apb_status apb_prefill(const apb_config* cfg, const void* q, const void* k, const void* v,
+                       const float* w1, const float* b1, const float* w2, const float* b2,
+                       void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  apb::Shape s;
+  apb_status st = check_config(cfg, &s);
+  if (st != APB_OK) return st;
+  if (!q || !k || !v || !w1 || !b1 || !w2 || !b2 || !out || !workspace)
+    return fail(APB_ERR_INVALID_ARG, "apb_prefill: NULL pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w1) || !aligned16(out) ||
+      !aligned16(workspace) || (lse && !aligned16(lse)))
+    return fail(APB_ERR_INVALID_ARG, "apb_prefill: pointers must be 16-byte aligned");
+  const PrefillLayout L = prefill_layout(s);
+  if (ws_bytes < L.total)
+    return fail(APB_ERR_INVALID_ARG, "apb_prefill: workspace %zu < %zu bytes", ws_bytes, L.total);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  auto* status = reinterpret_cast<apb::DeviceStatus*>(ws);
+  cudaError_t e = cudaMemsetAsync(&status->abort, 0, sizeof(uint32_t), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing abort flag");
+  const bool compress = s.H > 1 && s.keep > 0;
+  if (compress) {
+    // hosts 0..H-2 only: the last host's compressed block has no successor
+    apb::Shape s1 = s;
+    s1.H = s.H - 1;
+    s1.N = (long long)s1.H * s.n;
+    float* scores = reinterpret_cast<float*>(ws + L.scores);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+    const char* why = nullptr;
+    e = apb::launch_score(s1, q, k, v, w1, b1, w2, b2, scores, ws + L.wsplit, nullptr, status, cs,
+                          &why);
+    if (why) return fail(APB_ERR_CUDA, "score: %s", why);
+    if (e != cudaSuccess) return cuda_fail(e, "score kernel");
+    e = apb::launch_topk(s1, scores, idx, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k kernel");
+    e = apb::launch_gather(s1, k, v, idx, ws + L.pass_k, ws + L.pass_v, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "gather kernel");
+  }
+  apb::HostRange r{0, s.H, 0, 0, 0, s.N, s.N};
+  const char* why = nullptr;
+  e = apb::launch_attention(s, r, q, k, v, compress ? ws + L.pass_k : nullptr,
+                            compress ? ws + L.pass_v : nullptr, out, lse, status, cs, &why);
+  if (why) return fail(APB_ERR_CUDA, "attention: %s", why);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
+  return APB_OK;
+}
+
 apb_status apb_device_status(void* workspace, void* stream, int clear) {
   if (!workspace) return fail(APB_ERR_INVALID_ARG, "apb_device_status: NULL workspace");
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);

@@ -35,6 +35,27 @@ def host_range(n_hosts: int, rank: int, world: int) -> Tuple[int, int]:
     return rank * per, (rank + 1) * per
 
 
+def kv_head_range(n_kv_heads: int, rank: int, world: int) -> Tuple[int, int]:
+    """Kv heads owned by `rank` in the kv-head partitioning (the other natural
+    split of this path: every (host, kv head) unit is independent, so each
+    GPU runs the whole path on its kv heads and their q heads, with no
+    collective at all)."""
+    if n_kv_heads % world != 0:
+        raise ValueError(f"{n_kv_heads} kv heads do not split evenly over {world} ranks")
+    per = n_kv_heads // world
+    return rank * per, (rank + 1) * per
+
+
+def head_slice(x: dict, n_q_heads: int, n_kv_heads: int, gb: int, ge: int) -> dict:
+    """The inputs of kv heads [gb, ge) and their q heads, contiguous."""
+    G = n_q_heads // n_kv_heads
+    out = {"q": x["q"][:, gb * G:ge * G].contiguous(), "k": x["k"][:, gb:ge].contiguous(),
+           "v": x["v"][:, gb:ge].contiguous()}
+    for w in ("w1", "b1", "w2", "b2"):
+        out[w] = x[w][gb:ge].contiguous()
+    return out
+
+
 def nccl_all_gather(group=None) -> Callable[[torch.Tensor, torch.Tensor], None]:
     """In-place all-gather of a rank's chunk into the full buffer (NCCL):
     `chunk` must be this rank's slice of `full`."""

@@ -99,3 +99,16 @@ def test_selftest_argument_checks():
     assert apb._lib.apb_selftest_wait_timeout(FAKE, 64, 1000, None) == apb.APB_ERR_INVALID_ARG
     assert apb._lib.apb_selftest_wait_timeout(FAKE, 256, 0, None) == apb.APB_ERR_INVALID_ARG
     assert apb._lib.apb_selftest_wait_timeout(FAKE, 256, 2_000_000, None) == apb.APB_ERR_INVALID_ARG
+
+
+def test_prefill_workspace_and_checks():
+    c = apb.make_config(inputs.LLAMA8B_128K)
+    H, n, hkv, keep, d = 8, 16384, 8, 2048, 128
+    r = lambda x: (x + 255) // 256 * 256
+    expect = (256 + r(hkv * 256 * 384 * 4) + r(hkv * 256 * 4) + r((H - 1) * n * hkv * 4)
+              + r((H - 1) * hkv * keep * 4) + 2 * r(H * keep * hkv * d * 2))
+    assert apb.prefill_workspace_bytes(c) == expect
+    st = apb._lib.apb_prefill(ctypes.byref(c), *([FAKE] * 7), None, None, FAKE, 1 << 40, None)
+    assert st == apb.APB_ERR_INVALID_ARG                  # out is NULL
+    st = apb._lib.apb_prefill(ctypes.byref(c), *([FAKE] * 8), None, FAKE, 256, None)
+    assert st == apb.APB_ERR_INVALID_ARG                  # workspace too small

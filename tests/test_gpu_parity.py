@@ -210,3 +210,28 @@ def test_random_shapes_every_row(apb, shape):
                            n_q_heads=hq, n_kv_heads=hkv, head_dim=d, seed=31 + H + n + keep,
                            rope_theta=1e4 if d == 128 else None, needles_per_host=1)
     _full_parity(apb, cfg)
+
+
+@pytest.mark.parametrize("cfg", [inputs.TINY,
+                                 inputs.TINY.replace(n_hosts=5, block_len=300, anchor_len=75,
+                                                     keep=33, n_q_heads=10, head_dim=128, seed=4),
+                                 inputs.TINY.replace(n_hosts=1, seed=6),
+                                 inputs.TINY.replace(keep=0, seed=7)],
+                         ids=["tiny", "ragged_g5", "one_host", "keep0"])
+def test_single_call_prefill_equals_three_calls(apb, cfg):
+    # apb_prefill skips the last host's compressed block; its output and LSE
+    # must equal the three-call path's bit for bit
+    x = inputs.generate(cfg)
+    xd = _to_dev(x)
+    c = apb.make_config(cfg)
+    w = (xd["w1"], xd["b1"], xd["w2"], xd["b2"])
+    run = apb.Prefill(c)
+    apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, idx=run.idx, workspace=run.workspace)
+    apb.build_passing(c, xd["k"], xd["v"], run.idx, run.pass_k, run.pass_v)
+    ref, ref_lse = apb.block_attention(c, xd["q"], xd["k"], xd["v"], run.pass_k, run.pass_v,
+                                       want_lse=True, workspace=run.workspace)
+    ws = torch.zeros(apb.prefill_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    out, lse = apb.prefill(c, xd["q"], xd["k"], xd["v"], *w, want_lse=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert apb.device_status(ws) == apb.APB_OK
+    assert torch.equal(out, ref) and torch.equal(lse, ref_lse)

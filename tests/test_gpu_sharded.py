@@ -46,3 +46,29 @@ def test_sharded_equals_single_gpu(cfg, world):
     for sp in ranks:
         assert apb.device_status(sp.workspace) == apb.APB_OK
     assert torch.equal(torch.cat(outs), ref)
+
+
+@pytest.mark.parametrize("world", [2])
+def test_kv_head_sharding_equals_single_gpu(world):
+    # kv-head partitioning: each rank runs the whole path on its kv heads and
+    # their q heads; the outputs are the matching head slices of the full run
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_sparse_apb_b200 import _lib as apb
+    from long_context_sparse_apb_b200.sharded import head_slice, kv_head_range
+
+    cfg = inputs.TINY
+    x = inputs.generate(cfg)
+    xd = {k: v.cuda() for k, v in x.items() if k != "needles"}
+    full = apb.Prefill(apb.make_config(cfg))
+    ref = full(xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"], xd["b2"]).clone()
+    G = cfg.group
+    for r in range(world):
+        gb, ge = kv_head_range(cfg.n_kv_heads, r, world)
+        loc = head_slice(xd, cfg.n_q_heads, cfg.n_kv_heads, gb, ge)
+        c = apb.make_config(cfg, n_q_heads=(ge - gb) * G, n_kv_heads=ge - gb)
+        run = apb.Prefill(c)
+        out = run(loc["q"], loc["k"], loc["v"], loc["w1"], loc["b1"], loc["w2"], loc["b2"])
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref[:, gb * G:ge * G])
+        assert torch.equal(run.idx, full.idx[:, gb:ge])
