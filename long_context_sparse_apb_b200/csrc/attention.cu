@@ -80,11 +80,11 @@ struct Layout {
   static constexpr int kK0 = 2 * kTile;         // K stages
   static constexpr int kV0 = kK0 + kKStages * kTile;   // V stages
   static constexpr int kBars = kV0 + kVStages * kTile;
-  static constexpr int kBytes = kBars + 256;
 };
-// Both head sizes request the d = 128 footprint so that one CTA runs per SM
-// (each CTA allocates all 512 TMEM columns).
-constexpr int kSmemBytes = Layout<128>::kBytes + 1024;
+// Both head sizes request the d = 128 footprint (+256 bytes of barriers,
+// +1024 of alignment slack) so that one CTA runs per SM (each CTA allocates
+// all 512 TMEM columns).
+constexpr int kSmemBytes = Layout<128>::kBars + 256 + 1024;
 
 struct Params {
   int H, n, A, keep, Hq, Hkv, G, n_ctas_per_host;

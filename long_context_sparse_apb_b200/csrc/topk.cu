@@ -16,7 +16,6 @@ namespace apb {
 namespace {
 
 constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSmemKeys = 48 * 1024;   // 192 KB of keys
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -56,7 +55,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
                                                         long long N, int Hkv, bool stage) {
   extern __shared__ uint32_t skeys[];
   __shared__ int hist[256];
-  __shared__ int warp_sums[33];
+  __shared__ int warp_sums[kThreads / 32 + 1];
   __shared__ uint32_t s_digit;
   __shared__ int s_above;
 

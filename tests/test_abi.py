@@ -112,3 +112,22 @@ def test_prefill_workspace_and_checks():
     assert st == apb.APB_ERR_INVALID_ARG                  # out is NULL
     st = apb._lib.apb_prefill(ctypes.byref(c), *([FAKE] * 8), None, FAKE, 256, None)
     assert st == apb.APB_ERR_INVALID_ARG                  # workspace too small
+
+
+def test_host_range_and_query_aware_checks():
+    c = apb.make_config(inputs.TINY)
+    args = [FAKE] * 6 + [None, FAKE, 256, None]
+    for hb, he in ((0, 0), (2, 1), (-1, 2), (0, 5)):
+        assert apb._lib.apb_block_attention_hosts(ctypes.byref(c), hb, he, *args) == \
+            apb.APB_ERR_INVALID_ARG
+    st = apb._lib.apb_block_attention_hosts(ctypes.byref(c), 1, 3, None, *([FAKE] * 5), None,
+                                            FAKE, 256, None)
+    assert st == apb.APB_ERR_INVALID_ARG                  # q is NULL
+    # the query-aware variant needs room for its bias next to the weight split
+    st = apb._lib.apb_score_compress_query_aware(ctypes.byref(c), *([FAKE] * 8), FAKE, FAKE,
+                                                 256 + 2 * 256 * 192 * 4, None)
+    assert st == apb.APB_ERR_INVALID_ARG
+    bad = apb.make_config(inputs.TINY, head_dim=80)
+    st = apb._lib.apb_score_compress_query_aware(ctypes.byref(bad), *([FAKE] * 8), FAKE, FAKE,
+                                                 1 << 30, None)
+    assert st == apb.APB_ERR_UNSUPPORTED

@@ -235,3 +235,22 @@ def test_single_call_prefill_equals_three_calls(apb, cfg):
     torch.cuda.synchronize()
     assert apb.device_status(ws) == apb.APB_OK
     assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
+
+
+def test_topk_unstaged_path_large_block(apb):
+    # blocks above 48K tokens re-read their scores from global memory in every
+    # radix pass instead of staging them in shared memory
+    cfg = inputs.APBConfig("bigblock", n_hosts=2, block_len=50_000, anchor_len=0, query_len=0,
+                           keep=3000, n_q_heads=2, n_kv_heads=1, head_dim=64, seed=17)
+    x = inputs.generate(cfg)
+    xd = _to_dev(x)
+    c = apb.make_config(cfg)
+    scores = torch.empty((1, cfg.seq_len), dtype=torch.float32, device="cuda")
+    idx, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"],
+                                xd["b2"], scores=scores)
+    pk, pv = apb.build_passing(c, xd["k"], xd["v"], idx)
+    torch.cuda.synchronize()
+    s_ref = oracle_scores(cfg, x)
+    assert np.abs(scores.cpu().numpy() - s_ref).max() <= SCORE_ABS
+    check_topk(idx.cpu().numpy(), s_ref, cfg)
+    _check_passing_exact(x, idx.cpu().numpy(), pk, pv)
