@@ -96,10 +96,11 @@ size_t apb_workspace_bytes(const apb_config* cfg);
  *   idx [H, Hkv, keep] int32 (out): global positions, ascending per (h, g)
  *   workspace/ws_bytes: apb_workspace_bytes(cfg) bytes, or, when scores is
  *   given, the status block and the weight split only.
- * The products run on the tensor cores in bf16 with fp32 accumulation on an
- * exact rewrite: each fp32 weight is split into bf16 hi + lo, and the group
- * mean is folded into the q weights (W1_q / G applied to every q head), so
- * the only rounding beyond fp32 is the 2^-17 relative residual of the split. */
+ * The products run on the tensor cores in bf16 with fp32 accumulation on
+ * split operands: each fp32 weight is split into bf16 hi + lo, and the group
+ * mean of q (summed in fp32, then scaled by 1/G) likewise; k and v are exact
+ * bf16 and multiply both weight parts, the q mean as hi.hi + hi.lo + lo.hi.
+ * The rounding beyond fp32 is about 2^-17 relative per product. */
 apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* k,
                               const void* v, const float* w1, const float* b1,
                               const float* w2, const float* b2, float* scores,

@@ -4,25 +4,28 @@
 //     s[g,t] = w2[g] . SiLU(W1[g] x + b1[g]) + b2[g]
 //
 // The product W1 x must be fp32-accurate (the top-k that follows orders the
-// scores), while the tensor cores multiply bf16.  Two exact rewrites make that
-// possible:
-//   * the group mean is folded into the weights: W1_q (1/G) sum_j q_j =
-//     sum_j (W1_q / G) q_j, so every input row is an exact bf16 row of K, V or
-//     one q head, and no averaged (inexact) q ever exists;
-//   * each fp32 weight w is split into bf16 hi + lo (hi = rn(w), lo = rn(w -
-//     hi)), leaving |w - hi - lo| <= 2^-17 |w|; both halves are multiplied
-//     with fp32 accumulation.
-// So Z = X W1^T is computed as sum over the 2 + G input blocks of
-// X_b (Wh_b + Wl_b)^T with UMMA (M = 128 tokens, N = 256 hidden, K = 16),
-// accumulated in TMEM, and the epilogue applies b1, SiLU, w2 and b2 in fp32.
+// scores), while the tensor cores multiply bf16.  Every operand is therefore
+// split into bf16 parts whose products are accumulated in fp32:
+//   * each fp32 weight w into hi + lo (hi = rn(w), lo = rn(w - hi)), leaving
+//     |w - hi - lo| <= 2^-17 |w|;
+//   * k and v are exact bf16 and multiply both weight parts;
+//   * the group mean qbar (fp32 sum of G bf16 values, divided by G) into
+//     qh + ql the same way, multiplied as qh.Wh + qh.Wl + ql.Wh (the dropped
+//     ql.Wl term is below 2^-16 of the product).
+// So Z = X W1^T takes 2 + 2 + 3 UMMA groups per 16 input features instead of
+// one, with UMMA M = 128 tokens, N = 256 hidden, K = 16 accumulating in TMEM;
+// the epilogue applies b1, SiLU, w2 and b2 in fp32.
 //
 // split_weights_kernel writes Wh, Wl ([Hkv, 2, hidden, 3d] bf16) into the
 // workspace once per call.  score_kernel: one CTA = 256 tokens (two M = 128
-// accumulators, TMEM columns [0,256) and [256,512)) of one kv head; warp 8
-// streams B tiles (Wh, Wl of one 64-feature chunk, 2 x 32 KB, 2 stages) and
-// A tiles (128 tokens x 64 features of K, V or a q head, 16 KB, 4 stages)
-// with TMA; warp 9 issues the UMMAs; warps 0-7 run the epilogue, one token
-// row per thread.  Waits are bounded like the attention kernel's.
+// accumulators, TMEM columns [0,256) and [256,512)) of one kv head.  A
+// 4-slot ring of A tiles (128 tokens x 64 features, 16 KB) is filled by TMA
+// (warp 8) for the k and v features and, for the q features, by warps 0-7,
+// which read the group's q heads from global memory, form qbar in fp32 and
+// write qh and ql in the 128-byte-swizzled layout UMMA reads; warp 8 also
+// streams the B tiles (Wh, Wl of one 64-feature chunk, 2 x 32 KB, 2 stages);
+// warp 9 issues the UMMAs; warps 0-7 then run the epilogue, one token row per
+// thread.  Waits are bounded like the attention kernel's.
 #include <cuda_bf16.h>
 
 #include "apb_internal.h"
@@ -46,20 +49,24 @@ constexpr int kSmemBytes = kSmemBars + 256 + 2 * kHid * 4 + 1024;
 constexpr int kThreads = 320;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
-enum Bar { A_FULL = 0, A_EMPTY = 4, B_FULL = 8, B_EMPTY = 10, ACC_FULL = 12, DRAIN = 13, NUM = 14 };
+// HANDOFF: the producer has issued its last A load.  A converter waiting on
+// A_EMPTY before that could see the parity of a phase two completions old
+// (its first use of a slot is the slot's third) and overwrite a k or v tile.
+enum Bar {
+  A_FULL = 0, A_EMPTY = 4, B_FULL = 8, B_EMPTY = 10, ACC_FULL = 12, DRAIN = 13, HANDOFF = 14,
+  NUM = 15
+};
 
 __global__ void __launch_bounds__(256) split_weights_kernel(const float* __restrict__ w1,
                                                             __nv_bfloat16* __restrict__ ws,
-                                                            int Hkv, int F, int d, int G) {
+                                                            int Hkv, int F) {
   const long long per_head = (long long)kHid * F;
   const long long total = (long long)Hkv * per_head;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const long long g = i / per_head;
     const long long rem = i - g * per_head;
-    const int f = (int)(rem % F);
-    float w = w1[i];
-    if (f >= 2 * d) w = __fdiv_rn(w, (float)G);   // group mean folded in (exact for G = 2^k)
+    const float w = w1[i];
     const __nv_bfloat16 hi = __float2bfloat16_rn(w);
     const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
     ws[(2 * g) * per_head + rem] = hi;
@@ -99,6 +106,7 @@ __global__ void __launch_bounds__(256) query_bias_kernel(const __nv_bfloat16* __
 struct ScoreParams {
   long long N;
   int Hq, Hkv, G, d, F, n_chunks;
+  const __nv_bfloat16* q;
   const float* b1;
   const float* w2;
   const float* b2;
@@ -106,10 +114,81 @@ struct ScoreParams {
   DeviceStatus* status;
 };
 
-// A tiles of one chunk: 1 input block for k and v chunks, G for q chunks,
-// each for both 128-token halves.
-__device__ __forceinline__ int chunk_blocks(int c, int d, int G) {
-  return (c * kChunk) / d < 2 ? 1 : G;
+// Section of feature chunk c: 0 k, 1 v, 2 q.  A k or v chunk takes one A
+// tile per 128-token half (by TMA); a q chunk two (qh, ql) per half.
+__device__ __forceinline__ int chunk_section(int c, int d) { return (c * kChunk) / d; }
+
+// q features [off, off + 64) of one 128-token tile, in warps 0-7: thread tid
+// forms the group mean of 8 features (16 bytes of a row) for the 4 tokens
+// tid / 8 + 32 i, in fp32, and splits it into bf16 hi + lo.
+struct QTile {
+  uint32_t hi[4][4], lo[4][4];
+};
+
+__device__ __forceinline__ void q_tile_mean(const ScoreParams& p, long long row0, int g, int off,
+                                            float invG, QTile& o) {
+  const int tid = threadIdx.x;
+  const int piece = tid & 7;
+  const int rbase = tid >> 3;
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+  const long long head_stride = (long long)p.d;               // elements
+  const long long row_stride = (long long)p.Hq * p.d;
+  const __nv_bfloat16* base = p.q + (long long)g * p.G * head_stride + off + piece * 8;
+#pragma unroll 1
+  for (int j0 = 0; j0 < p.G; j0 += 4) {
+    uint4 raw[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const long long t = row0 + rbase + 32 * i;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        raw[i][u] = make_uint4(0u, 0u, 0u, 0u);
+        if (t < p.N && j0 + u < p.G)
+          raw[i][u] = __ldg(reinterpret_cast<const uint4*>(base + t * row_stride +
+                                                           (long long)(j0 + u) * head_stride));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {raw[i][u].x, raw[i][u].y, raw[i][u].z, raw[i][u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[i][2 * e] += __uint_as_float(w[e] << 16);
+          acc[i][2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+        }
+      }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = acc[i][2 * e] * invG, x1 = acc[i][2 * e + 1] * invG;
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+      const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
+      o.hi[i][e] = *reinterpret_cast<const uint32_t*>(&h);
+      o.lo[i][e] = *reinterpret_cast<const uint32_t*>(&l);
+    }
+}
+
+// Writes a QTile into two A slots in the 128-byte-swizzled K-major layout
+// UMMA reads (16-byte chunk index XOR row % 8 inside each 1024-byte group of
+// 8 rows: what a TMA load with 128-byte swizzle would have written).
+__device__ __forceinline__ void q_tile_store(const QTile& o, uint8_t* slot_h, uint8_t* slot_l) {
+  const int piece = threadIdx.x & 7;
+  const int rbase = threadIdx.x >> 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = rbase + 32 * i;
+    const int at = r * 128 + ((piece ^ (r & 7)) << 4);
+    *reinterpret_cast<uint4*>(slot_h + at) = make_uint4(o.hi[i][0], o.hi[i][1], o.hi[i][2], o.hi[i][3]);
+    *reinterpret_cast<uint4*>(slot_l + at) = make_uint4(o.lo[i][0], o.lo[i][1], o.lo[i][2], o.lo[i][3]);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -129,6 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = blockIdx.y;
   const long long t0 = (long long)blockIdx.x * (2 * kTile);
   const volatile uint32_t* gabort = &p.status->abort;
+  const int q_chunk0 = 2 * p.d / kChunk;      // first chunk of the q section
+  const int q_slot0 = 2 * q_chunk0;           // its first A slot (k and v: 2 per chunk)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM; ++i) ptx::mbar_init(&bars[i], 1);
@@ -160,6 +241,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !skip) {
+      // the q rows the converters read, into L2 ahead of them
+      for (int c = q_chunk0; c < p.n_chunks; ++c)
+        for (int j = 0; j < p.G; ++j)
+          for (int m = 0; m < 2; ++m)
+            ptx::tma_prefetch_l2_3d(&mQ, c * kChunk - 2 * p.d, g * p.G + j,
+                                    (int)(t0 + m * kTile));
       int lastA[kAStages] = {-1, -1, -1, -1}, lastB[kBStages] = {-1, -1};
       int ai = 0;
       bool ok = true;
@@ -175,30 +262,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tma_load_3d(bdst, &mW, &bars[B_FULL + bs], c * kChunk, 0, 2 * g);
         ptx::tma_load_3d(bdst + kBHalf, &mW, &bars[B_FULL + bs], c * kChunk, 0, 2 * g + 1);
         lastB[bs] = (int)bpar;
-        const int sec = (c * kChunk) / p.d;
-        const int off = c * kChunk - sec * p.d;
-        const int nb = chunk_blocks(c, p.d, p.G);
-        for (int b = 0; b < nb && ok; ++b) {
-          for (int m = 0; m < 2; ++m, ++ai) {
-            const int as = ai % kAStages;
-            const uint32_t apar = (ai / kAStages) & 1;
-            if (!ptx::mbar_wait_bounded(&bars[A_EMPTY + as], apar ^ 1, gabort, kWaitLimitNs)) {
-              record_failure(p.status, 72, ai);
-              ok = false;
-              break;
-            }
-            uint8_t* adst = smem + kSmemA + as * kATile;
-            const int row = (int)(t0 + m * kTile);
-            ptx::mbar_arrive_expect_tx(&bars[A_FULL + as], kATile);
-            if (sec == 0)
-              ptx::tma_load_3d(adst, &mK, &bars[A_FULL + as], off, g, row);
-            else if (sec == 1)
-              ptx::tma_load_3d(adst, &mV, &bars[A_FULL + as], off, g, row);
-            else
-              ptx::tma_load_3d(adst, &mQ, &bars[A_FULL + as], off, g * p.G + b, row);
-            lastA[as] = (int)apar;
-          }
+        const int sec = chunk_section(c, p.d);
+        if (sec == 2) {       // q slots are filled by the converter warps
+          ai += 4;
+          continue;
         }
+        const int off = c * kChunk - sec * p.d;
+        for (int m = 0; m < 2; ++m, ++ai) {
+          const int as = ai % kAStages;
+          const uint32_t apar = (ai / kAStages) & 1;
+          if (!ptx::mbar_wait_bounded(&bars[A_EMPTY + as], apar ^ 1, gabort, kWaitLimitNs)) {
+            record_failure(p.status, 72, ai);
+            ok = false;
+            break;
+          }
+          uint8_t* adst = smem + kSmemA + as * kATile;
+          const int row = (int)(t0 + m * kTile);
+          ptx::mbar_arrive_expect_tx(&bars[A_FULL + as], kATile);
+          ptx::tma_load_3d(adst, sec == 0 ? &mK : &mV, &bars[A_FULL + as], off, g, row);
+          lastA[as] = (int)apar;
+        }
+        if (ok && c == q_chunk0 - 1) ptx::mbar_arrive(&bars[HANDOFF]);
       }
       for (int s = 0; s < kAStages; ++s)
         if (lastA[s] >= 0) ptx::mbar_wait_bounded(&bars[A_FULL + s], lastA[s], never, kWaitLimitNs);
@@ -221,31 +305,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        const int nb = chunk_blocks(c, p.d, p.G);
-        for (int b = 0; b < nb && ok; ++b) {
-          for (int m = 0; m < 2; ++m, ++ai) {
-            const int as = ai % kAStages;
-            if (!ptx::mbar_wait_bounded(&bars[A_FULL + as], (ai / kAStages) & 1, gabort,
+        const uint32_t bh = aB + bs * 2 * kBHalf, bl = bh + kBHalf;
+        const bool qsec = chunk_section(c, p.d) == 2;
+        for (int m = 0; m < 2 && ok; ++m) {
+          // k, v: one A slot (x, exact bf16); q: two (qh, ql)
+          const int nslots = qsec ? 2 : 1;
+          for (int u = 0; u < nslots; ++u) {
+            const int as = (ai + u) % kAStages;
+            if (!ptx::mbar_wait_bounded(&bars[A_FULL + as], ((ai + u) / kAStages) & 1, gabort,
                                         kWaitLimitNs)) {
-              record_failure(p.status, 75, ai);
+              record_failure(p.status, 75, ai + u);
               ok = false;
-              break;
             }
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < kChunk / 16; ++ks) {
-#pragma unroll
-              for (int part = 0; part < 2; ++part) {
-                ptx::umma_bf16_ss(tmem + 256 * m,
-                                  ptx::sdesc_sw128(aA + as * kATile + ks * 32, 16, 1024),
-                                  ptx::sdesc_sw128(aB + bs * 2 * kBHalf + part * kBHalf + ks * 32,
-                                                   16, 1024),
-                                  idesc, started[m] ? 1u : 0u);
-                started[m] = true;
-              }
-            }
-            ptx::umma_commit(&bars[A_EMPTY + as]);
+            if (!ok) break;
           }
+          if (!ok) break;
+          ptx::tc_fence_after();
+          const uint32_t ah = aA + (ai % kAStages) * kATile;
+          const uint32_t al = aA + ((ai + 1) % kAStages) * kATile;
+          const uint32_t acc = tmem + 256 * m;
+#pragma unroll
+          for (int ks = 0; ks < kChunk / 16; ++ks) {
+            const uint64_t dAh = ptx::sdesc_sw128(ah + ks * 32, 16, 1024);
+            const uint64_t dBh = ptx::sdesc_sw128(bh + ks * 32, 16, 1024);
+            const uint64_t dBl = ptx::sdesc_sw128(bl + ks * 32, 16, 1024);
+            ptx::umma_bf16_ss(acc, dAh, dBh, idesc, started[m] ? 1u : 0u);
+            started[m] = true;
+            ptx::umma_bf16_ss(acc, dAh, dBl, idesc, 1u);
+            if (qsec)
+              ptx::umma_bf16_ss(acc, ptx::sdesc_sw128(al + ks * 32, 16, 1024), dBh, idesc, 1u);
+          }
+          for (int u = 0; u < nslots; ++u) ptx::umma_commit(&bars[A_EMPTY + (ai + u) % kAStages]);
+          ai += nslots;
         }
         if (ok) ptx::umma_commit(&bars[B_EMPTY + bs]);
       }
@@ -254,7 +345,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_wait_bounded(&bars[DRAIN], 0, never, kWaitLimitNs);
     }
   } else if (!skip) {
-    // ------------------------------------------------------------ epilogue
+    // ---------------------------------------------- q converters, then epilogue
+    {
+      const float invG = 1.0f / (float)p.G;     // exact for G = 2^k
+      int ai = q_slot0;
+      for (int c = q_chunk0; c < p.n_chunks; ++c) {
+        bool ok = true;
+        for (int m = 0; m < 2; ++m, ai += 2) {
+          const int sh = ai % kAStages, sl = (ai + 1) % kAStages;
+          const uint32_t par = ((ai / kAStages) & 1) ^ 1;
+          // loads first: their latency overlaps the wait for the slots
+          QTile qt;
+          q_tile_mean(p, t0 + m * kTile, g, c * kChunk - 2 * p.d, invG, qt);
+          if (threadIdx.x == 0) {
+            ok = (ai != q_slot0 ||
+                  ptx::mbar_wait_bounded(&bars[HANDOFF], 0, gabort, kWaitLimitNs)) &&
+                 ptx::mbar_wait_bounded(&bars[A_EMPTY + sh], par, gabort, kWaitLimitNs) &&
+                 ptx::mbar_wait_bounded(&bars[A_EMPTY + sl], par, gabort, kWaitLimitNs);
+            if (!ok) record_failure(p.status, 77, ai);
+          }
+          ok = ptx::barrier_and(1, 256, ok);
+          if (!ok) break;
+          q_tile_store(qt, smem + kSmemA + sh * kATile, smem + kSmemA + sl * kATile);
+          ptx::fence_proxy_async_smem();
+          ptx::named_barrier_sync(1, 256);
+          if (threadIdx.x == 0) {
+            ptx::mbar_arrive(&bars[A_FULL + sh]);
+            ptx::mbar_arrive(&bars[A_FULL + sl]);
+          }
+        }
+        if (!ok) break;
+      }
+    }
     const int m = warp >> 2;                        // token half
     const int row = threadIdx.x & 127;
     const uint32_t taddr = tmem + 256 * m + ((uint32_t)((warp & 3) * 32) << 16);
@@ -300,7 +422,7 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   split_weights_kernel<<<sms * 4, 256, 0, st>>>(w1, static_cast<__nv_bfloat16*>(wsplit), s.Hkv,
-                                                F, s.d, G);
+                                                F);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -332,6 +454,7 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
   p.G = G;
   p.d = s.d;
   p.F = F;
+  p.q = static_cast<const __nv_bfloat16*>(q);
   // the query-aware variant stops after the k and v sections: its q section
   // is a per-head constant already folded into qbias
   p.n_chunks = (qbias ? 2 * s.d : F) / kChunk;
