@@ -13,49 +13,82 @@
 //     qh + ql the same way, multiplied as qh.Wh + qh.Wl + ql.Wh (the dropped
 //     ql.Wl term is below 2^-16 of the product).
 // So Z = X W1^T takes 2 + 2 + 3 UMMA groups per 16 input features instead of
-// one, with UMMA M = 128 tokens, N = 256 hidden, K = 16 accumulating in TMEM;
-// the epilogue applies b1, SiLU, w2 and b2 in fp32.
+// one; the epilogue applies b1, SiLU, w2 and b2 in fp32.
 //
 // split_weights_kernel writes Wh, Wl ([Hkv, 2, hidden, 3d] bf16) into the
-// workspace once per call.  score_kernel: one CTA = 256 tokens (two M = 128
-// accumulators, TMEM columns [0,256) and [256,512)) of one kv head.  A
-// 4-slot ring of A tiles (128 tokens x 64 features, 16 KB) is filled by TMA
-// (warp 8) for the k and v features and, for the q features, by warps 0-7,
-// which read the group's q heads from global memory, form qbar in fp32 and
-// write qh and ql in the 128-byte-swizzled layout UMMA reads; warp 8 also
-// streams the B tiles (Wh, Wl of one 64-feature chunk, 2 x 32 KB, 2 stages);
-// warp 9 issues the UMMAs; warps 0-7 then run the epilogue, one token row per
-// thread.  Waits are bounded like the attention kernel's.
+// workspace once per call.  score_kernel is persistent and runs on CTA pairs
+// (clusters of 2, one per TPC): a tile is 256 tokens of one kv head, 128 per
+// CTA, and one tcgen05.mma.cta_group::2 of M = 256 tokens, N = 256 hidden,
+// K = 16 covers the pair, so each CTA stages only its 128 tokens and its 128
+// hidden rows of Wh / Wl.  The pair's even CTA issues every UMMA; the
+// accumulators are double-buffered in TMEM (2 x 256 columns), so the
+// epilogue of tile i runs under the UMMAs of tile i + 1.  Per CTA:
+//   warp 14    TMA producer of the k and v tiles (128 tokens x 64 features,
+//              16 KB, 4-slot ring);
+//   warp 12    TMA producer of the Wh / Wl halves of a 64-feature chunk
+//              (2 x 16 KB, 3 stages);
+//   warps 4-11 q converters: read the group's G q heads from global memory
+//              (the loads in flight sit in their registers), form qbar in
+//              fp32 and write qh, ql (2-pair ring) in the 128-byte-swizzled
+//              K-major layout UMMA reads;
+//   warp 13    UMMA issuer (even CTA) / TMEM allocation (both);
+//   warps 0-3  epilogue, one token row per thread.
+// Full barriers live in the even CTA and count both CTAs' arrivals; empty
+// barriers live in both and get one commit each.  Waits are bounded like the
+// attention kernel's.
 #include <cuda_bf16.h>
 
 #include "apb_internal.h"
 #include "device_status.cuh"
+#include "sm100_pair.cuh"
 #include "sm100_ptx.cuh"
 
 namespace apb {
 namespace {
 
 constexpr int kHid = 256;
-constexpr int kTile = 128;                 // tokens per accumulator
+constexpr int kTile = 128;                 // tokens per CTA and tile (the pair: 256)
+constexpr int kHalf = kHid / 2;            // hidden rows of B per CTA
 constexpr int kChunk = 64;                 // features per chunk (128-byte rows)
-constexpr int kAStages = 4;
-constexpr int kBStages = 2;
+constexpr int kKVStages = 4;
+constexpr int kQStages = 2;                // (qh, ql) pairs
+constexpr int kBStages = 3;
 constexpr int kATile = kTile * kChunk * 2;          // 16 KB
-constexpr int kBHalf = kHid * kChunk * 2;           // 32 KB (hi or lo)
-constexpr int kSmemA = 0;
-constexpr int kSmemB = kAStages * kATile;           // 64 KB
-constexpr int kSmemBars = kSmemB + kBStages * 2 * kBHalf;   // 192 KB
-constexpr int kSmemBytes = kSmemBars + 256 + 2 * kHid * 4 + 1024;
-constexpr int kThreads = 320;
+constexpr int kBPart = kHalf * kChunk * 2;          // 16 KB (hi or lo half)
+constexpr int kSmemKV = 0;
+constexpr int kSmemQ = kSmemKV + kKVStages * kATile;          // 64 KB
+constexpr int kSmemB = kSmemQ + kQStages * 2 * kATile;        // 128 KB
+constexpr int kSmemBars = kSmemB + kBStages * 2 * kBPart;     // 224 KB
+constexpr int kSmemB1 = kSmemBars + 256;                     // b1, w2 of the current head
+// The tiles need 1024-byte alignment; the dynamic shared memory of this
+// kernel (which has no static shared memory) starts at such an address, and
+// the kernel checks that instead of reserving slack for it.
+constexpr int kSmemBytes = kSmemB1 + 2 * kHid * 4;
+constexpr int kEpiThreads = 128;           // warps 0-3
+constexpr int kConvThreads = 256;          // warps 4-11
+constexpr int kBWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kKVWarp = 14;
+constexpr int kThreads = 480;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint64_t kDrainLimitNs = 100000000ull;
 
-// HANDOFF: the producer has issued its last A load.  A converter waiting on
-// A_EMPTY before that could see the parity of a phase two completions old
-// (its first use of a slot is the slot's third) and overwrite a k or v tile.
+// Full barriers (KV_FULL, Q_FULL, B_FULL) and ACC_EMPTY are used in the even
+// CTA only, with 2 arrivals per phase (one per CTA); the others get one
+// arrival (a UMMA commit) in each CTA.
 enum Bar {
-  A_FULL = 0, A_EMPTY = 4, B_FULL = 8, B_EMPTY = 10, ACC_FULL = 12, DRAIN = 13, HANDOFF = 14,
-  NUM = 15
+  KV_FULL = 0,
+  KV_EMPTY = KV_FULL + kKVStages,
+  Q_FULL = KV_EMPTY + kKVStages,
+  Q_EMPTY = Q_FULL + kQStages,
+  B_FULL = Q_EMPTY + kQStages,
+  B_EMPTY = B_FULL + kBStages,
+  ACC_FULL = B_EMPTY + kBStages,
+  ACC_EMPTY = ACC_FULL + 2,
+  DRAIN = ACC_EMPTY + 2,
+  NUM = DRAIN + 1
 };
+static_assert(NUM * 8 + 8 <= 256, "barriers and the TMEM address fit their 256 bytes");
 
 __global__ void __launch_bounds__(256) split_weights_kernel(const float* __restrict__ w1,
                                                             __nv_bfloat16* __restrict__ ws,
@@ -106,6 +139,7 @@ __global__ void __launch_bounds__(256) query_bias_kernel(const __nv_bfloat16* __
 struct ScoreParams {
   long long N;
   int Hq, Hkv, G, d, F, n_chunks;
+  int tiles_per_head, n_tiles;       // tiles of 256 tokens
   const __nv_bfloat16* q;
   const float* b1;
   const float* w2;
@@ -114,118 +148,137 @@ struct ScoreParams {
   DeviceStatus* status;
 };
 
-// Section of feature chunk c: 0 k, 1 v, 2 q.  A k or v chunk takes one A
-// tile per 128-token half (by TMA); a q chunk two (qh, ql) per half.
+// Section of feature chunk c: 0 k, 1 v, 2 q.
 __device__ __forceinline__ int chunk_section(int c, int d) { return (c * kChunk) / d; }
 
-// q features [off, off + 64) of one 128-token tile, in warps 0-7: thread tid
-// forms the group mean of 8 features (16 bytes of a row) for the 4 tokens
-// tid / 8 + 32 i, in fp32, and splits it into bf16 hi + lo.
-struct QTile {
-  uint32_t hi[4][4], lo[4][4];
+// The q section of the CTA's 128 tokens, every q chunk at once, in two
+// passes of 64 tokens (warps 4-11).  In pass sp, thread ct takes the 16-byte
+// piece ct % 8 (8 features) of every q chunk for the tokens
+// sp * 64 + ct / 8 + 32 i, i < 2, and reads it from the group's G heads, 4
+// heads at a time: the 8 lanes of a token cover a whole 128-byte line per
+// load, and a pass reads each token's G * d * 2 contiguous bytes.  The sums
+// run in fp32; the mean (x 1/G) is split into bf16 hi + lo.
+constexpr int kMaxQChunks = 2;             // d <= 128
+
+struct QLoad {
+  uint4 v[kMaxQChunks][2][4];              // [chunk][token][head of the group]
+};
+struct QAcc {
+  float a[kMaxQChunks][2][8];              // [chunk][token][feature]
 };
 
-__device__ __forceinline__ void q_tile_mean(const ScoreParams& p, long long row0, int g, int off,
-                                            float invG, QTile& o) {
-  const int tid = threadIdx.x;
-  const int piece = tid & 7;
-  const int rbase = tid >> 3;
-  float acc[4][8];
+__device__ __forceinline__ void q_issue(const ScoreParams& p, long long row0, int g, int sp,
+                                        int j0, int n_q, int ct, QLoad& L) {
+  const int piece = ct & 7;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i) {
+    const long long t = row0 + sp * 64 + (ct >> 3) + 32 * i;
+    const __nv_bfloat16* base =
+        p.q + t * ((long long)p.Hq * p.d) + (long long)(g * p.G + j0) * p.d + piece * 8;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
-  const long long head_stride = (long long)p.d;               // elements
-  const long long row_stride = (long long)p.Hq * p.d;
-  const __nv_bfloat16* base = p.q + (long long)g * p.G * head_stride + off + piece * 8;
-#pragma unroll 1
-  for (int j0 = 0; j0 < p.G; j0 += 4) {
-    uint4 raw[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const long long t = row0 + rbase + 32 * i;
+    for (int c = 0; c < kMaxQChunks; ++c)
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        raw[i][u] = make_uint4(0u, 0u, 0u, 0u);
-        if (t < p.N && j0 + u < p.G)
-          raw[i][u] = __ldg(reinterpret_cast<const uint4*>(base + t * row_stride +
-                                                           (long long)(j0 + u) * head_stride));
+        L.v[c][i][u] = make_uint4(0u, 0u, 0u, 0u);
+        if (c < n_q && t < p.N && j0 + u < p.G)
+          L.v[c][i][u] =
+              __ldg(reinterpret_cast<const uint4*>(base + (long long)u * p.d + c * kChunk));
       }
-    }
+  }
+}
+
+__device__ __forceinline__ void q_accumulate(const QLoad& L, QAcc& A) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+  for (int c = 0; c < kMaxQChunks; ++c)
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const uint32_t w[4] = {raw[i][u].x, raw[i][u].y, raw[i][u].z, raw[i][u].w};
+        const uint32_t w[4] = {L.v[c][i][u].x, L.v[c][i][u].y, L.v[c][i][u].z, L.v[c][i][u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          acc[i][2 * e] += __uint_as_float(w[e] << 16);
-          acc[i][2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+          A.a[c][i][2 * e] += __uint_as_float(w[e] << 16);
+          A.a[c][i][2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
         }
       }
-  }
+}
+
+// Splits a pass's sums (x 1/G) into bf16 hi + lo and writes them into the
+// (qh, ql) slot pair of each q chunk, in the 128-byte-swizzled K-major
+// layout UMMA reads (16-byte chunk index XOR row % 8 inside each 1024-byte
+// group of 8 rows: what a TMA load with 128-byte swizzle would have written).
+// Piece by piece, so no second copy of the pass is held in registers.
+__device__ __forceinline__ void q_split_store(const QAcc& A, float invG, int sp, int n_q, int ct,
+                                              uint8_t* qbase, int qu) {
+  const int piece = ct & 7;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int c = 0; c < kMaxQChunks; ++c) {
+    if (c >= n_q) break;
+    uint8_t* slot = qbase + ((qu + c) % kQStages) * 2 * kATile;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float x0 = acc[i][2 * e] * invG, x1 = acc[i][2 * e + 1] * invG;
-      const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-      const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
-      o.hi[i][e] = *reinterpret_cast<const uint32_t*>(&h);
-      o.lo[i][e] = *reinterpret_cast<const uint32_t*>(&l);
+    for (int i = 0; i < 2; ++i) {
+      const int r = sp * 64 + (ct >> 3) + 32 * i;
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = A.a[c][i][2 * e] * invG, x1 = A.a[c][i][2 * e + 1] * invG;
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+        const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
+        hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[e] = *reinterpret_cast<const uint32_t*>(&l);
+      }
+      const int at = r * 128 + ((piece ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(slot + at) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(slot + kATile + at) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-}
-
-// Writes a QTile into two A slots in the 128-byte-swizzled K-major layout
-// UMMA reads (16-byte chunk index XOR row % 8 inside each 1024-byte group of
-// 8 rows: what a TMA load with 128-byte swizzle would have written).
-__device__ __forceinline__ void q_tile_store(const QTile& o, uint8_t* slot_h, uint8_t* slot_l) {
-  const int piece = threadIdx.x & 7;
-  const int rbase = threadIdx.x >> 3;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = rbase + 32 * i;
-    const int at = r * 128 + ((piece ^ (r & 7)) << 4);
-    *reinterpret_cast<uint4*>(slot_h + at) = make_uint4(o.hi[i][0], o.hi[i][1], o.hi[i][2], o.hi[i][3]);
-    *reinterpret_cast<uint4*>(slot_l + at) = make_uint4(o.lo[i][0], o.lo[i][1], o.lo[i][2], o.lo[i][3]);
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(512, 1)   // 512: caps registers at 128 (launched with 480)
     score_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                  const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mW,
                  const ScoreParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((ptx::smem_u32(smem) & 1023u) != 0u) {      // same in both CTAs of the pair
+    if (threadIdx.x == 0) record_failure(p.status, 90, 0);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBars);
+  float* s_b1 = reinterpret_cast<float*>(smem + kSmemB1);
+  float* s_w2 = s_b1 + kHid;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + NUM);
   uint32_t* s_flags = s_tmem + 1;
-  float* s_b1 = reinterpret_cast<float*>(smem + kSmemBars + 256);
-  float* s_w2 = s_b1 + kHid;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = blockIdx.y;
-  const long long t0 = (long long)blockIdx.x * (2 * kTile);
+  const uint32_t rank = pair::cta_rank();
+  const int cl = (int)pair::cluster_id_x(), ncl = (int)pair::n_clusters_x();
   const volatile uint32_t* gabort = &p.status->abort;
   const int q_chunk0 = 2 * p.d / kChunk;      // first chunk of the q section
-  const int q_slot0 = 2 * q_chunk0;           // its first A slot (k and v: 2 per chunk)
+  const int n_q = p.n_chunks - q_chunk0;      // q chunks per tile (0: query-aware)
+  // A tile's chunks run q first, then k, v: the converters then have the whole
+  // k and v part of a tile to prepare the next tile's q.
+  auto chunk_at = [&](int i) { return i < n_q ? q_chunk0 + i : i - n_q; };
+  // the token rows of this CTA in tile t, and its kv head
+  auto tile_g = [&](int t) { return t / p.tiles_per_head; };
+  auto tile_row = [&](int t) {
+    return (long long)(t % p.tiles_per_head) * (2 * kTile) + (long long)rank * kTile;
+  };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NUM; ++i) ptx::mbar_init(&bars[i], 1);
+    for (int i = 0; i < NUM; ++i) {
+      const bool two = (i < KV_EMPTY) || (i >= Q_FULL && i < Q_EMPTY) ||
+                       (i >= B_FULL && i < B_EMPTY) || (i >= ACC_EMPTY && i < DRAIN);
+      ptx::mbar_init(&bars[i], two ? 2 : 1);
+    }
     ptx::fence_mbar_init();
     s_flags[0] = *gabort;
     s_flags[1] = 0u;
   }
-  if (threadIdx.x < kHid) {
-    s_b1[threadIdx.x] = p.b1[g * kHid + threadIdx.x];
-    s_w2[threadIdx.x] = p.w2[g * kHid + threadIdx.x];
+  if (warp == kMmaWarp) {
+    pair::tmem_alloc(s_tmem, 512);
+    pair::tmem_relinquish();
   }
-  if (warp == 9) {
-    ptx::tmem_alloc(s_tmem, 512);
-    ptx::tmem_relinquish();
-  }
-  if (warp == 8 && lane == 0) {
+  if (warp == kBWarp && lane == 0) {
     ptx::tma_prefetch_desc(&mQ);
     ptx::tma_prefetch_desc(&mK);
     ptx::tma_prefetch_desc(&mV);
@@ -233,180 +286,255 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   ptx::tc_fence_before();
   __syncthreads();
+  pair::cluster_sync();       // barriers of both CTAs initialised before any arrival
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const volatile uint32_t* never = s_flags + 1;
   const bool skip = s_flags[0] != 0u;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
+  if (warp == kBWarp || warp == kKVWarp) {
+    // ------------------------------------------------------------ producers
+    // Two threads, so that neither ring waits on the other: warp 12 streams
+    // the B halves (every chunk), warp 14 the k and v tiles (k, v chunks).
     if (lane == 0 && !skip) {
-      // the q rows the converters read, into L2 ahead of them
-      for (int c = q_chunk0; c < p.n_chunks; ++c)
-        for (int j = 0; j < p.G; ++j)
-          for (int m = 0; m < 2; ++m)
-            ptx::tma_prefetch_l2_3d(&mQ, c * kChunk - 2 * p.d, g * p.G + j,
-                                    (int)(t0 + m * kTile));
-      int lastA[kAStages] = {-1, -1, -1, -1}, lastB[kBStages] = {-1, -1};
-      int ai = 0;
+      const bool isB = warp == kBWarp;
+      const int stages = isB ? kBStages : kKVStages;
+      uint64_t* full = &bars[isB ? B_FULL : KV_FULL];
+      uint64_t* empty = &bars[isB ? B_EMPTY : KV_EMPTY];
+      int u = 0;
       bool ok = true;
-      for (int c = 0; c < p.n_chunks && ok; ++c) {
-        const int bs = c & 1;
-        const uint32_t bpar = (c >> 1) & 1;
-        if (!ptx::mbar_wait_bounded(&bars[B_EMPTY + bs], bpar ^ 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 70 + bs, c);
-          break;
-        }
-        uint8_t* bdst = smem + kSmemB + bs * 2 * kBHalf;
-        ptx::mbar_arrive_expect_tx(&bars[B_FULL + bs], 2 * kBHalf);
-        ptx::tma_load_3d(bdst, &mW, &bars[B_FULL + bs], c * kChunk, 0, 2 * g);
-        ptx::tma_load_3d(bdst + kBHalf, &mW, &bars[B_FULL + bs], c * kChunk, 0, 2 * g + 1);
-        lastB[bs] = (int)bpar;
-        const int sec = chunk_section(c, p.d);
-        if (sec == 2) {       // q slots are filled by the converter warps
-          ai += 4;
-          continue;
-        }
-        const int off = c * kChunk - sec * p.d;
-        for (int m = 0; m < 2; ++m, ++ai) {
-          const int as = ai % kAStages;
-          const uint32_t apar = (ai / kAStages) & 1;
-          if (!ptx::mbar_wait_bounded(&bars[A_EMPTY + as], apar ^ 1, gabort, kWaitLimitNs)) {
-            record_failure(p.status, 72, ai);
+      for (int t = cl; t < p.n_tiles && ok; t += ncl) {
+        const int g = tile_g(t);
+        const int row = (int)tile_row(t);
+        for (int i = 0; i < p.n_chunks; ++i) {
+          const int c = chunk_at(i);
+          const int sec = chunk_section(c, p.d);
+          if (!isB && sec == 2) continue;       // q tiles come from the converters
+          const int s = u % stages;
+          if (!ptx::mbar_wait_bounded(&empty[s], ((u / stages) & 1) ^ 1, gabort, kWaitLimitNs)) {
+            record_failure(p.status, (isB ? 80 : 82) + rank, u);
             ok = false;
             break;
           }
-          uint8_t* adst = smem + kSmemA + as * kATile;
-          const int row = (int)(t0 + m * kTile);
-          ptx::mbar_arrive_expect_tx(&bars[A_FULL + as], kATile);
-          ptx::tma_load_3d(adst, sec == 0 ? &mK : &mV, &bars[A_FULL + as], off, g, row);
-          lastA[as] = (int)apar;
+          const uint32_t fc = pair::map_to(&full[s], 0);
+          if (isB) {
+            uint8_t* dst = smem + kSmemB + s * 2 * kBPart;
+            pair::arrive_expect_tx_remote(fc, 2 * kBPart);
+            pair::tma_load_3d(dst, &mW, fc, c * kChunk, (int)rank * kHalf, 2 * g);
+            pair::tma_load_3d(dst + kBPart, &mW, fc, c * kChunk, (int)rank * kHalf, 2 * g + 1);
+          } else {
+            pair::arrive_expect_tx_remote(fc, kATile);
+            pair::tma_load_3d(smem + kSmemKV + s * kATile, sec == 0 ? &mK : &mV, fc,
+                              c * kChunk - sec * p.d, g, row);
+          }
+          ++u;
         }
-        if (ok && c == q_chunk0 - 1) ptx::mbar_arrive(&bars[HANDOFF]);
       }
-      for (int s = 0; s < kAStages; ++s)
-        if (lastA[s] >= 0) ptx::mbar_wait_bounded(&bars[A_FULL + s], lastA[s], never, kWaitLimitNs);
-      for (int s = 0; s < kBStages; ++s)
-        if (lastB[s] >= 0) ptx::mbar_wait_bounded(&bars[B_FULL + s], lastB[s], never, kWaitLimitNs);
+      // copies in flight land before the CTA may exit: wait until the UMMAs
+      // have released the last use of every slot (bounded; on a failure the
+      // copies have long completed when the limit passes)
+      for (int v = u - stages; v < u; ++v)
+        if (v >= 0)
+          ptx::mbar_wait_bounded(&empty[v % stages], (v / stages) & 1, never,
+                                 ok ? kWaitLimitNs : kDrainLimitNs);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !skip) {
-      const uint32_t idesc = ptx::idesc_bf16_f32(kTile, kHid, 0);
-      const uint32_t aA = ptx::smem_u32(smem + kSmemA);
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0 && rank == 0 && !skip) {
+      const uint32_t idesc = ptx::idesc_bf16_f32(2 * kTile, kHid, 0);
+      const uint32_t aKV = ptx::smem_u32(smem + kSmemKV);
+      const uint32_t aQ = ptx::smem_u32(smem + kSmemQ);
       const uint32_t aB = ptx::smem_u32(smem + kSmemB);
-      bool started[2] = {false, false};
-      int ai = 0;
+      // a commit tracks every UMMA issued before it; one to each CTA's barrier
+      auto commit_both = [&](int bar) {
+        pair::umma_commit(pair::map_to(&bars[bar], 0));
+        pair::umma_commit(pair::map_to(&bars[bar], 1));
+      };
+      int kvu = 0, qu = 0, bu = 0, it = 0;
       bool ok = true;
-      for (int c = 0; c < p.n_chunks && ok; ++c) {
-        const int bs = c & 1;
-        if (!ptx::mbar_wait_bounded(&bars[B_FULL + bs], (c >> 1) & 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 74, c);
+      for (int t = cl; t < p.n_tiles && ok; t += ncl, ++it) {
+        const int b = it & 1;
+        if (!pair::spin_cluster_bounded(&bars[ACC_EMPTY + b], ((it >> 1) & 1) ^ 1, gabort,
+                                        kWaitLimitNs)) {
+          record_failure(p.status, 84, it);
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t bh = aB + bs * 2 * kBHalf, bl = bh + kBHalf;
-        const bool qsec = chunk_section(c, p.d) == 2;
-        for (int m = 0; m < 2 && ok; ++m) {
-          // k, v: one A slot (x, exact bf16); q: two (qh, ql)
-          const int nslots = qsec ? 2 : 1;
-          for (int u = 0; u < nslots; ++u) {
-            const int as = (ai + u) % kAStages;
-            if (!ptx::mbar_wait_bounded(&bars[A_FULL + as], ((ai + u) / kAStages) & 1, gabort,
-                                        kWaitLimitNs)) {
-              record_failure(p.status, 75, ai + u);
-              ok = false;
-            }
-            if (!ok) break;
+        const uint32_t acc = tmem + 256 * b;
+        bool first = true;
+        for (int i = 0; i < p.n_chunks && ok; ++i) {
+          const int c = chunk_at(i);
+          const int bs = bu % kBStages;
+          const bool qsec = chunk_section(c, p.d) == 2;
+          const int s = qsec ? qu % kQStages : kvu % kKVStages;
+          ok = pair::spin_cluster_bounded(&bars[B_FULL + bs], (bu / kBStages) & 1, gabort,
+                                          kWaitLimitNs) &&
+               (qsec ? pair::spin_cluster_bounded(&bars[Q_FULL + s], (qu / kQStages) & 1, gabort,
+                                                  kWaitLimitNs)
+                     : pair::spin_cluster_bounded(&bars[KV_FULL + s], (kvu / kKVStages) & 1,
+                                                  gabort, kWaitLimitNs));
+          if (!ok) {
+            record_failure(p.status, 85, c);
+            break;
           }
-          if (!ok) break;
           ptx::tc_fence_after();
-          const uint32_t ah = aA + (ai % kAStages) * kATile;
-          const uint32_t al = aA + ((ai + 1) % kAStages) * kATile;
-          const uint32_t acc = tmem + 256 * m;
+          const uint32_t bh = aB + bs * 2 * kBPart, bl = bh + kBPart;
+          const uint32_t xh = qsec ? aQ + s * 2 * kATile : aKV + s * kATile;
+          const uint32_t xl = xh + kATile;     // ql (q chunks only)
 #pragma unroll
           for (int ks = 0; ks < kChunk / 16; ++ks) {
-            const uint64_t dAh = ptx::sdesc_sw128(ah + ks * 32, 16, 1024);
+            const uint64_t dXh = ptx::sdesc_sw128(xh + ks * 32, 16, 1024);
             const uint64_t dBh = ptx::sdesc_sw128(bh + ks * 32, 16, 1024);
             const uint64_t dBl = ptx::sdesc_sw128(bl + ks * 32, 16, 1024);
-            ptx::umma_bf16_ss(acc, dAh, dBh, idesc, started[m] ? 1u : 0u);
-            started[m] = true;
-            ptx::umma_bf16_ss(acc, dAh, dBl, idesc, 1u);
+            pair::umma_bf16_ss(acc, dXh, dBh, idesc, first ? 0u : 1u);
+            first = false;
+            pair::umma_bf16_ss(acc, dXh, dBl, idesc, 1u);
             if (qsec)
-              ptx::umma_bf16_ss(acc, ptx::sdesc_sw128(al + ks * 32, 16, 1024), dBh, idesc, 1u);
+              pair::umma_bf16_ss(acc, ptx::sdesc_sw128(xl + ks * 32, 16, 1024), dBh, idesc, 1u);
           }
-          for (int u = 0; u < nslots; ++u) ptx::umma_commit(&bars[A_EMPTY + (ai + u) % kAStages]);
-          ai += nslots;
+          commit_both(qsec ? Q_EMPTY + s : KV_EMPTY + s);
+          commit_both(B_EMPTY + bs);
+          ++bu;
+          if (qsec) ++qu; else ++kvu;
         }
-        if (ok) ptx::umma_commit(&bars[B_EMPTY + bs]);
+        if (ok) commit_both(ACC_FULL + b);
       }
-      if (ok) ptx::umma_commit(&bars[ACC_FULL]);
-      ptx::umma_commit(&bars[DRAIN]);
+      commit_both(DRAIN);
       ptx::mbar_wait_bounded(&bars[DRAIN], 0, never, kWaitLimitNs);
     }
-  } else if (!skip) {
-    // ---------------------------------------------- q converters, then epilogue
-    {
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ q converters
+    // Units of work: (tile, pass, group of 4 heads).  The loads of unit k + 1
+    // are issued before unit k is split and stored, so they are in flight
+    // while this thread waits for free slots and writes shared memory.
+    if (!skip && n_q > 0) {
+      const int ct = threadIdx.x - 128;
       const float invG = 1.0f / (float)p.G;     // exact for G = 2^k
-      int ai = q_slot0;
-      for (int c = q_chunk0; c < p.n_chunks; ++c) {
-        bool ok = true;
-        for (int m = 0; m < 2; ++m, ai += 2) {
-          const int sh = ai % kAStages, sl = (ai + 1) % kAStages;
-          const uint32_t par = ((ai / kAStages) & 1) ^ 1;
-          // loads first: their latency overlaps the wait for the slots
-          QTile qt;
-          q_tile_mean(p, t0 + m * kTile, g, c * kChunk - 2 * p.d, invG, qt);
-          if (threadIdx.x == 0) {
-            ok = (ai != q_slot0 ||
-                  ptx::mbar_wait_bounded(&bars[HANDOFF], 0, gabort, kWaitLimitNs)) &&
-                 ptx::mbar_wait_bounded(&bars[A_EMPTY + sh], par, gabort, kWaitLimitNs) &&
-                 ptx::mbar_wait_bounded(&bars[A_EMPTY + sl], par, gabort, kWaitLimitNs);
-            if (!ok) record_failure(p.status, 77, ai);
-          }
-          ok = ptx::barrier_and(1, 256, ok);
-          if (!ok) break;
-          q_tile_store(qt, smem + kSmemA + sh * kATile, smem + kSmemA + sl * kATile);
-          ptx::fence_proxy_async_smem();
-          ptx::named_barrier_sync(1, 256);
-          if (threadIdx.x == 0) {
-            ptx::mbar_arrive(&bars[A_FULL + sh]);
-            ptx::mbar_arrive(&bars[A_FULL + sl]);
-          }
+      const int ng = (p.G + 3) / 4;
+      const int my_tiles = cl < p.n_tiles ? (p.n_tiles - 1 - cl) / ncl + 1 : 0;
+      const int n_units = my_tiles * 2 * ng;
+      auto issue = [&](int k, QLoad& L) {
+        const int ti = k / (2 * ng), rem = k - ti * 2 * ng;
+        const int t = cl + ti * ncl;
+        q_issue(p, tile_row(t), tile_g(t), rem / ng, (rem % ng) * 4, n_q, ct, L);
+      };
+      QLoad L;
+      QAcc A;
+      if (n_units > 0) issue(0, L);
+      int qu = 0;                                // q pair uses so far (n_q per tile)
+      bool ok = true;
+      for (int k = 0; k < n_units && ok; ++k) {
+        const int rem = k % (2 * ng), sp = rem / ng, jg = rem % ng;
+        if (jg == 0) {
+#pragma unroll
+          for (int c = 0; c < kMaxQChunks; ++c)
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) A.a[c][pp][e] = 0.f;   // [chunk][token][feature]
         }
-        if (!ok) break;
+        q_accumulate(L, A);
+        if (k + 1 < n_units) issue(k + 1, L);   // in flight during the wait and the stores
+        if (jg != ng - 1) continue;
+        if (sp == 0) {          // the tile's slots, released by the UMMAs of the last use
+          if (ct == 0)
+            for (int c = 0; c < n_q && ok; ++c) {
+              const int u = qu + c;
+              ok = ptx::mbar_wait_bounded(&bars[Q_EMPTY + u % kQStages],
+                                          ((u / kQStages) & 1) ^ 1, gabort, kWaitLimitNs);
+              if (!ok) record_failure(p.status, 86 + rank, u);
+            }
+          ok = ptx::barrier_and(1, kConvThreads, ok);
+          if (!ok) break;
+        }
+        q_split_store(A, invG, sp, n_q, ct, smem + kSmemQ, qu);
+        if (sp == 1) {          // tile complete: publish its pairs to the issuer
+          ptx::fence_proxy_async_smem();
+          ptx::named_barrier_sync(1, kConvThreads);
+          if (ct == 0)
+            for (int c = 0; c < n_q; ++c)
+              pair::arrive_remote(pair::map_to(&bars[Q_FULL + (qu + c) % kQStages], 0));
+          qu += n_q;
+        }
       }
     }
-    const int m = warp >> 2;                        // token half
-    const int row = threadIdx.x & 127;
-    const uint32_t taddr = tmem + 256 * m + ((uint32_t)((warp & 3) * 32) << 16);
-    bool ok = ptx::mbar_wait_bounded(&bars[ACC_FULL], 0, gabort, kWaitLimitNs);
-    if (!__all_sync(0xffffffffu, ok)) {
-      if (lane == 0) record_failure(p.status, 76, m);
-    } else {
-      ptx::tc_fence_after();
-      float part = 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < kHid / 32; ++cc) {
-        uint32_t z[32];
-        APB_TMEM_LD32(taddr + 32 * cc, z);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float zz = __uint_as_float(z[x]) + s_b1[32 * cc + x];
-          const float silu = __fdividef(zz, 1.0f + __expf(-zz));
-          part = fmaf(s_w2[32 * cc + x], silu, part);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    if (!skip) {
+      const int row = threadIdx.x;                      // 0..127 = TMEM lane
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      int it = 0, cur_g = -1;
+      for (int t = cl; t < p.n_tiles; t += ncl, ++it) {
+        const int b = it & 1;
+        const int g = tile_g(t);
+        if (g != cur_g) {       // this head's b1, w2 into shared memory
+          ptx::named_barrier_sync(2, kEpiThreads);
+          for (int u = row; u < kHid; u += kEpiThreads) {
+            s_b1[u] = p.b1[g * kHid + u];
+            s_w2[u] = p.w2[g * kHid + u];
+          }
+          ptx::named_barrier_sync(2, kEpiThreads);
+          cur_g = g;
         }
+        const float4* b1 = reinterpret_cast<const float4*>(s_b1);
+        const float4* w2 = reinterpret_cast<const float4*>(s_w2);
+        const bool ok = ptx::mbar_wait_bounded(&bars[ACC_FULL + b], (it >> 1) & 1, gabort,
+                                               kWaitLimitNs);
+        if (!ptx::barrier_and(2, kEpiThreads, ok)) {
+          if (row == 0) record_failure(p.status, 88 + rank, it);
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t taddr = tmem + 256 * b + lane_off;
+        // column chunks of 32, the load of chunk cc + 1 in flight while
+        // chunk cc is evaluated (two register sets)
+        uint32_t z0[32], z1[32];
+        float part[4] = {0.f, 0.f, 0.f, 0.f};     // 4 chains: no serial FFMA latency
+        auto eval = [&](const uint32_t* z, int cc) {
+#pragma unroll
+          for (int x4 = 0; x4 < 8; ++x4) {
+            const float4 bb = b1[8 * cc + x4];
+            const float4 ww = w2[8 * cc + x4];
+            const float bv[4] = {bb.x, bb.y, bb.z, bb.w}, wv[4] = {ww.x, ww.y, ww.z, ww.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float zz = __uint_as_float(z[4 * x4 + e]) + bv[e];
+              const float silu = __fdividef(zz, 1.0f + __expf(-zz));
+              part[e] = fmaf(wv[e], silu, part[e]);
+            }
+          }
+        };
+        APB_TMEM_LD32_ASYNC(taddr, z0);
+        APB_TMEM_WAIT32(z0);
+#pragma unroll 1
+        for (int cc = 0; cc < kHid / 32; cc += 2) {
+          APB_TMEM_LD32_ASYNC(taddr + 32 * (cc + 1), z1);
+          eval(z0, cc);
+          APB_TMEM_WAIT32(z1);
+          if (cc + 2 < kHid / 32) APB_TMEM_LD32_ASYNC(taddr + 32 * (cc + 2), z0);
+          eval(z1, cc + 1);
+          if (cc + 2 < kHid / 32) APB_TMEM_WAIT32(z0);
+        }
+        // accumulator b read out by all 128 rows: hand it back to the issuer
+        ptx::tc_fence_before();
+        ptx::named_barrier_sync(2, kEpiThreads);
+        if (row == 0) pair::arrive_remote(pair::map_to(&bars[ACC_EMPTY + b], 0));
+        const long long tok = tile_row(t) + row;
+        if (tok < p.N)
+          p.scores[(long long)g * p.N + tok] = ((part[0] + part[1]) + (part[2] + part[3])) + __ldg(p.b2 + g);
       }
-      const long long t = t0 + m * kTile + row;
-      if (t < p.N) p.scores[(long long)g * p.N + t] = part + p.b2[g];
     }
   }
 
+  // Both CTAs stay resident until the pair is done: the even CTA's UMMAs read
+  // the odd CTA's shared memory, and the odd CTA arrives on the even one's
+  // barriers.
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  pair::cluster_sync();
+  if (warp == kMmaWarp) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 512);
+    pair::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -442,7 +570,7 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
             encode_bf16_3d(&mV, v, s.d, s.Hkv, N, (uint64_t)s.d * 2, (uint64_t)s.Hkv * s.d * 2, 64,
                            1, kTile) &&
             encode_bf16_3d(&mW, wsplit, F, kHid, (uint64_t)s.Hkv * 2, (uint64_t)F * 2,
-                           (uint64_t)kHid * F * 2, 64, kHid, 1);
+                           (uint64_t)kHid * F * 2, 64, kHalf, 1);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point or argument)";
     return cudaErrorInvalidValue;
@@ -463,11 +591,39 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
   p.b2 = b2;
   p.scores = scores;
   p.status = status;
+  p.tiles_per_head = (int)((s.N + 2 * kTile - 1) / (2 * kTile));
+  p.n_tiles = p.tiles_per_head * s.Hkv;
+  if (p.n_tiles == 0) return cudaSuccess;
   e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((s.N + 2 * kTile - 1) / (2 * kTile)), s.Hkv);
-  score_kernel<<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, mW, p);
-  return cudaGetLastError();
+
+  // persistent: as many CTA pairs as can be resident at once (once per device)
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = kSmemBytes;
+  lc.stream = st;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  static int resident_pairs[64] = {0};
+  int pairs = dev >= 0 && dev < 64 ? resident_pairs[dev] : 0;
+  if (pairs == 0) {
+    lc.gridDim = dim3(2 * (sms / 2));
+    e = cudaOccupancyMaxActiveClusters(&pairs, score_kernel, &lc);
+    if (e != cudaSuccess) return e;
+    if (pairs < 1) {
+      *why = "score kernel: no CTA pair fits on the device";
+      return cudaErrorInvalidConfiguration;
+    }
+    if (dev >= 0 && dev < 64) resident_pairs[dev] = pairs;
+  }
+  if (pairs > p.n_tiles) pairs = p.n_tiles;
+  lc.gridDim = dim3(2 * pairs);
+  return cudaLaunchKernelEx(&lc, score_kernel, mQ, mK, mV, mW, p);
 }
 
 }  // namespace apb
