@@ -319,11 +319,11 @@ __global__ void __launch_bounds__(512, 1)   // 512: caps registers at 128 (launc
           const uint32_t fc = pair::map_to(&full[s], 0);
           if (isB) {
             uint8_t* dst = smem + kSmemB + s * 2 * kBPart;
-            pair::arrive_expect_tx_remote(fc, 2 * kBPart);
+            pair::arrive_expect_tx_relaxed(fc, 2 * kBPart);
             pair::tma_load_3d(dst, &mW, fc, c * kChunk, (int)rank * kHalf, 2 * g);
             pair::tma_load_3d(dst + kBPart, &mW, fc, c * kChunk, (int)rank * kHalf, 2 * g + 1);
           } else {
-            pair::arrive_expect_tx_remote(fc, kATile);
+            pair::arrive_expect_tx_relaxed(fc, kATile);
             pair::tma_load_3d(smem + kSmemKV + s * kATile, sec == 0 ? &mK : &mV, fc,
                               c * kChunk - sec * p.d, g, row);
           }

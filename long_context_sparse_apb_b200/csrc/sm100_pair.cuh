@@ -57,6 +57,18 @@ __device__ __forceinline__ void arrive_expect_tx_remote(uint32_t bar_cluster, ui
       : "memory");
 }
 
+// The same without release semantics: for a producer whose arrival publishes
+// no memory writes of its own (the bytes of its TMA loads are counted by the
+// barrier itself), so the thread is not held until its earlier accesses are
+// visible across the cluster.
+__device__ __forceinline__ void arrive_expect_tx_relaxed(uint32_t bar_cluster, uint32_t bytes) {
+  asm volatile(
+      "mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+          bar_cluster),
+      "r"(bytes)
+      : "memory");
+}
+
 // Phase wait with acquire at cluster scope (the arrivals come from both CTAs).
 __device__ __forceinline__ bool try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
