@@ -468,10 +468,11 @@ def attention_variants(apb, cfg, xd, dev, stream, apb_ms, reps=3):
 
 
 def run_sharded(args, cfg):
-    """One sequence prefilled by N GPUs, hosts split evenly (the pages'
-    distributed form): per step each rank compresses its hosts, the compressed
-    blocks are all-gathered over NCCL, each rank attends its hosts.  Strong
-    scaling: value = tokens of the one sequence / max-over-ranks step time."""
+    """One sequence prefilled by N GPUs, hosts split evenly and round-robin
+    (the pages' distributed form; round-robin balances the per-host work):
+    per step each rank compresses its hosts, the compressed blocks are
+    all-gathered over NCCL, each rank attends its hosts.  Strong scaling:
+    value = tokens of the one sequence / max-over-ranks step time."""
     from long_context_sparse_apb_b200 import _lib as apb
     from long_context_sparse_apb_b200.sharded import ShardedPrefill, nccl_all_gather
 
@@ -480,7 +481,8 @@ def run_sharded(args, cfg):
     c = apb.make_config(cfg)
     sp = ShardedPrefill(c, rank, world, device=dev,
                         all_gather=nccl_all_gather() if world > 1 else None)
-    loc = {k: v.to(dev) for k, v in inputs.generate_local(cfg, sp.hb, sp.he).items()}
+    loc = {k: v.to(dev) for k, v in inputs.generate_local(
+        cfg, sp.first, sp.first + sp.count * sp.stride, sp.stride).items()}
     w = (loc["w1"], loc["b1"], loc["w2"], loc["b2"])
     stream = torch.cuda.current_stream(dev)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -521,14 +523,14 @@ def run_sharded(args, cfg):
               for name, a, b in (("compress", 0, 1), ("exchange", 1, 2), ("attention", 2, 3))}
     if rank == 0:
         cdict = config_dict(cfg, world)
-        cdict["parallelism"] = (f"host-sharded: {world} GPU(s) x {cfg.n_hosts // world} host(s), "
-                                f"NCCL all-gather of the compressed blocks")
+        cdict["parallelism"] = (f"host-sharded: {world} GPU(s) x {cfg.n_hosts // world} host(s) "
+                                f"({sp.order}), NCCL all-gather of the compressed blocks")
         line = {"metric": METRIC, "value": cfg.seq_len / (max_ms / 1e3 / args.steps),
                 "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": max_ms / args.steps, "higher_is_better": True,
                 "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": cdict, "stages_ms_max_over_ranks": stages,
-                "exchange_bytes_per_rank": 2 * (sp.he - sp.hb) * cfg.keep * cfg.n_kv_heads
+                "exchange_bytes_per_rank": 2 * sp.count * cfg.keep * cfg.n_kv_heads
                 * cfg.head_dim * 2,
                 "e2e": None, "e2e_note": "host-buffer end-to-end is measured in the default mode",
                 "gpu_launches": args.steps * (cfg.n_hosts // world) * (4 if cfg.keep else 2)

@@ -173,6 +173,26 @@ apb_status apb_block_attention_hosts(const apb_config* cfg, int32_t host_begin, 
                                      const void* pass_k, const void* pass_v, void* out,
                                      float* lse, void* workspace, size_t ws_bytes, void* stream);
 
+/* Step 3 for an evenly spaced set of hosts on rank-local buffers: the hosts
+ * host_first + i*host_stride, i < host_count (main features: hosts are spread
+ * over devices; a round-robin assignment, rank r of W owning hosts r, r+W,
+ * ..., balances the work, which grows with the host index because each host
+ * attends to the compressed blocks of all hosts before it).  Same
+ * computation and buffer conventions as apb_block_attention_hosts, with the
+ * set's hosts in increasing order in place of a contiguous range:
+ *   q, out  [host_count*n, Hq, d]; kv_k, kv_v [A + host_count*n, Hkv, d]
+ *   (anchor rows, then the hosts' rows); pass_k, pass_v [H*keep, Hkv, d] in
+ *   host order (rows [0, h_last*keep) are read); lse [Hq, host_count*n].
+ * host_first >= 0, host_count >= 1, host_stride >= 1 and
+ * host_first + (host_count-1)*host_stride < n_hosts, else
+ * APB_ERR_INVALID_ARG.  apb_block_attention_hosts(b, e) is this call with
+ * (b, e - b, 1). */
+apb_status apb_block_attention_host_set(const apb_config* cfg, int32_t host_first,
+                                        int32_t host_count, int32_t host_stride, const void* q,
+                                        const void* kv_k, const void* kv_v, const void* pass_k,
+                                        const void* pass_v, void* out, float* lse,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
 /* The whole path in one call: steps 1-3 on one GPU for all hosts, writing
  * out [N, Hq, d] (and lse [Hq, N] when not NULL).  The last host's
  * compressed block is not computed: no host follows it, so no passing block

@@ -52,6 +52,9 @@ _lib.apb_block_attention.restype = ctypes.c_int
 _lib.apb_block_attention_hosts.argtypes = ([ctypes.POINTER(Config), ctypes.c_int32, ctypes.c_int32]
                                            + [_P] * 8 + [ctypes.c_size_t, _P])
 _lib.apb_block_attention_hosts.restype = ctypes.c_int
+_lib.apb_block_attention_host_set.argtypes = ([ctypes.POINTER(Config)] + [ctypes.c_int32] * 3
+                                              + [_P] * 8 + [ctypes.c_size_t, _P])
+_lib.apb_block_attention_host_set.restype = ctypes.c_int
 _lib.apb_score_compress_static.argtypes = [ctypes.POINTER(Config)] + [_P] * 9
 _lib.apb_score_compress_static.restype = ctypes.c_int
 _lib.apb_score_compress_static_max_floats.argtypes = []
@@ -269,6 +272,42 @@ def block_attention_hosts(c: Config, host_begin: int, host_end: int, q, kv_k, kv
                                         _ptr(pass_v) if use_pass else None, _ptr(out), _ptr(lse),
                                         _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "apb_block_attention_hosts")
+    return out, lse
+
+
+def block_attention_host_set(c: Config, host_first: int, host_count: int, host_stride: int, q,
+                             kv_k, kv_v, pass_k, pass_v, out=None, lse=None, want_lse=False,
+                             workspace=None, stream=None):
+    """apb_block_attention_host_set: attention of the hosts host_first +
+    i*host_stride, i < host_count, on rank-local buffers (q/out: those hosts'
+    rows in order; kv_k/kv_v: the anchor's rows, then those hosts' rows).
+    Returns (out, lse or None)."""
+    _, hq, hkv, d = _dims(c)
+    rows = host_count * c.block_len
+    _want(q, "q", torch.bfloat16, (rows, hq, d))
+    _want(kv_k, "kv_k", torch.bfloat16, (c.anchor_len + rows, hkv, d))
+    _want(kv_v, "kv_v", torch.bfloat16, (c.anchor_len + rows, hkv, d))
+    use_pass = c.keep > 0 and host_first + (host_count - 1) * host_stride >= 1
+    if use_pass:
+        shape = (c.n_hosts * c.keep, hkv, d)
+        _want(pass_k, "pass_k", torch.bfloat16, shape)
+        _want(pass_v, "pass_v", torch.bfloat16, shape)
+    if out is None:
+        out = torch.empty((rows, hq, d), dtype=torch.bfloat16, device=q.device)
+    _want(out, "out", torch.bfloat16, (rows, hq, d))
+    if lse is None and want_lse:
+        lse = torch.empty((hq, rows), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (hq, rows))
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    st = _lib.apb_block_attention_host_set(ctypes.byref(c), host_first, host_count, host_stride,
+                                           _ptr(q), _ptr(kv_k), _ptr(kv_v),
+                                           _ptr(pass_k) if use_pass else None,
+                                           _ptr(pass_v) if use_pass else None, _ptr(out),
+                                           _ptr(lse), _ptr(workspace), workspace.numel(),
+                                           _stream(stream))
+    _check(st, "apb_block_attention_host_set")
     return out, lse
 
 

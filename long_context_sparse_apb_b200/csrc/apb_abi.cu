@@ -157,20 +157,26 @@ apb_status apb_build_passing(const apb_config* cfg, const void* k, const void* v
   return APB_OK;
 }
 
-static apb_status attention_impl(const char* who, const apb_config* cfg, int hb, int he,
-                                 bool local, const void* q, const void* k, const void* v,
+// Attention of the hosts h0, h0 + stride, ..., h0 + (count - 1) * stride.
+// local: rank-local buffers (Q/out hold those hosts' rows in that order; K/V
+// the anchor rows, then the hosts' rows); else whole-sequence buffers (then
+// stride must be 1).
+static apb_status attention_impl(const char* who, const apb_config* cfg, int h0, int count,
+                                 int stride, bool local, const void* q, const void* k, const void* v,
                                  const void* pass_k, const void* pass_v, void* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream) {
   apb::Shape s;
   apb_status st = check_config(cfg, &s);
   if (st != APB_OK) return st;
-  if (hb < 0 || he > s.H || hb >= he)
-    return fail(APB_ERR_INVALID_ARG, "%s: host range [%d, %d) not inside [0, %d)", who, hb, he,
-                s.H);
+  if (h0 < 0 || count < 1 || stride < 1 || (!local && stride != 1) ||
+      (long long)h0 + (long long)(count - 1) * stride >= s.H)
+    return fail(APB_ERR_INVALID_ARG, "%s: hosts %d + i*%d, i < %d, not inside [0, %d)", who, h0,
+                stride, count, s.H);
+  const int h_last = h0 + (count - 1) * stride;
   if (!q || !k || !v || !out || !workspace)
     return fail(APB_ERR_INVALID_ARG, "%s: NULL q/k/v/out/workspace", who);
   // hosts h >= 1 read pass rows [0, h*keep)
-  const bool need_pass = s.keep > 0 && he > 1;
+  const bool need_pass = s.keep > 0 && h_last >= 1;
   if (need_pass && (!pass_k || !pass_v))
     return fail(APB_ERR_INVALID_ARG, "%s: NULL pass_k/pass_v with keep > 0", who);
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace) ||
@@ -180,19 +186,20 @@ static apb_status attention_impl(const char* who, const apb_config* cfg, int hb,
     return fail(APB_ERR_INVALID_ARG, "%s: workspace %zu < %zu bytes", who, ws_bytes,
                 apb::kStatusBytes);
   apb::HostRange r;
-  r.hb = hb;
-  r.he = he;
+  r.h0 = h0;
+  r.count = count;
+  r.stride = stride;
   if (local) {
-    // rank-local buffers: Q/out hold hosts [hb, he); K/V hold the anchor rows
+    // rank-local buffers: Q/out hold the hosts' rows; K/V hold the anchor rows
     // [0, A) followed by those hosts' rows
     r.q_row0 = 0;
     r.k_row0 = s.A;
     r.anchor_row0 = 0;
-    r.q_rows = (long long)(he - hb) * s.n;
+    r.q_rows = (long long)count * s.n;
     r.k_rows = s.A + r.q_rows;
   } else {
-    r.q_row0 = hb * s.n;
-    r.k_row0 = hb * s.n;
+    r.q_row0 = h0 * s.n;
+    r.k_row0 = h0 * s.n;
     r.anchor_row0 = 0;
     r.q_rows = s.N;
     r.k_rows = s.N;
@@ -215,16 +222,27 @@ apb_status apb_block_attention(const apb_config* cfg, const void* q, const void*
                                void* out, float* lse, void* workspace, size_t ws_bytes,
                                void* stream) {
   const int H = cfg ? cfg->n_hosts : 1;
-  return attention_impl("apb_block_attention", cfg, 0, H, false, q, k, v, pass_k, pass_v, out, lse,
-                        workspace, ws_bytes, stream);
+  return attention_impl("apb_block_attention", cfg, 0, H, 1, false, q, k, v, pass_k, pass_v, out,
+                        lse, workspace, ws_bytes, stream);
 }
 
 apb_status apb_block_attention_hosts(const apb_config* cfg, int32_t host_begin, int32_t host_end,
                                      const void* q, const void* kv_k, const void* kv_v,
                                      const void* pass_k, const void* pass_v, void* out,
                                      float* lse, void* workspace, size_t ws_bytes, void* stream) {
-  return attention_impl("apb_block_attention_hosts", cfg, host_begin, host_end, true, q, kv_k,
-                        kv_v, pass_k, pass_v, out, lse, workspace, ws_bytes, stream);
+  return attention_impl("apb_block_attention_hosts", cfg, host_begin, host_end - host_begin, 1,
+                        true, q, kv_k, kv_v, pass_k, pass_v, out, lse, workspace, ws_bytes,
+                        stream);
+}
+
+apb_status apb_block_attention_host_set(const apb_config* cfg, int32_t host_first,
+                                        int32_t host_count, int32_t host_stride, const void* q,
+                                        const void* kv_k, const void* kv_v, const void* pass_k,
+                                        const void* pass_v, void* out, float* lse,
+                                        void* workspace, size_t ws_bytes, void* stream) {
+  return attention_impl("apb_block_attention_host_set", cfg, host_first, host_count, host_stride,
+                        true, q, kv_k, kv_v, pass_k, pass_v, out, lse, workspace, ws_bytes,
+                        stream);
 }
 
 // ---------------------------------------------------------------- one call
@@ -292,7 +310,7 @@ apb_status apb_prefill(const apb_config* cfg, const void* q, const void* k, cons
     e = apb::launch_gather(s1, k, v, idx, ws + L.pass_k, ws + L.pass_v, cs);
     if (e != cudaSuccess) return cuda_fail(e, "gather kernel");
   }
-  apb::HostRange r{0, s.H, 0, 0, 0, s.N, s.N};
+  apb::HostRange r{0, s.H, 1, 0, 0, 0, s.N, s.N};
   const char* why = nullptr;
   e = apb::launch_attention(s, r, q, k, v, compress ? ws + L.pass_k : nullptr,
                             compress ? ws + L.pass_v : nullptr, out, lse, status, cs, &why);

@@ -53,8 +53,11 @@ cudaError_t launch_gather(const Shape& s, const void* k, const void* v, const in
 // Hosts [hb, he) of one attention launch and where their rows sit: row of
 // host hb's first token in the Q/out buffer (q_row0) and in the K/V buffer
 // (k_row0), row of the anchor's first token in K/V, and the buffers' rows.
+// The hosts h0, h0 + stride, ..., h0 + (count - 1) * stride of one attention
+// launch, whose rows sit one after another (in that order) in the Q/out and
+// K/V buffers from q_row0 and k_row0; the anchor's rows start at anchor_row0.
 struct HostRange {
-  int hb, he, q_row0, k_row0, anchor_row0;
+  int h0, count, stride, q_row0, k_row0, anchor_row0;
   long long q_rows, k_rows;
 };
 

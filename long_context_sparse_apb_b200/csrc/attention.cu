@@ -88,9 +88,10 @@ constexpr int kSmemBytes = Layout<128>::kBars + 256 + 1024;
 
 struct Params {
   int H, n, A, keep, Hq, Hkv, G, n_ctas_per_host;
-  // hosts [hb, he) of this launch; rows, in the Q/out and K/V buffers, of the
-  // first token of host hb, and, in K/V, of the anchor's first token
-  int hb, he, q_row0, k_row0, anchor_row0;
+  // hosts h0 + i * hstride, i < hcount, of this launch, one after another in
+  // the Q/out and K/V buffers from rows q_row0 / k_row0; the anchor's first
+  // token at K/V row anchor_row0
+  int h0, hcount, hstride, q_row0, k_row0, anchor_row0;
   long long N;   // rows of the Q/out buffer (the lse row stride)
   float scale_log2;
   __nv_bfloat16* out;
@@ -139,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // heavy units first: the last query tiles of the last hosts
   const int u = p.n_ctas_per_host - 1 - (int)blockIdx.x;
   const int head = (int)blockIdx.y;
-  const int h = p.he - 1 - (int)blockIdx.z;
+  const int li = p.hcount - 1 - (int)blockIdx.z;   // launch-local host index
+  const int h = p.h0 + li * p.hstride;
   const int g = head / p.G;
   const int qA0 = 2 * u * kRows;                 // first local row of tile A
   const int na = (h >= 1 && p.A > 0) ? (p.A + kRows - 1) / kRows : 0;
@@ -148,8 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int TA = na + np + 2 * u + 1;            // KV tiles of query tile A
   const int TB = (qA0 + kRows < p.n) ? TA + 1 : 0;   // of tile B (0: beyond the block)
   const int Tmax = TB > 0 ? TB : TA;
-  const int local_row0 = p.k_row0 + (h - p.hb) * p.n;   // K/V row of this host's token 0
-  const int q_row0 = p.q_row0 + (h - p.hb) * p.n;       // Q/out row of this host's token 0
+  const int local_row0 = p.k_row0 + li * p.n;   // K/V row of this host's token 0
+  const int q_row0 = p.q_row0 + li * p.n;       // Q/out row of this host's token 0
 
   const volatile uint32_t* gabort = &p.status->abort;
 
@@ -499,8 +501,9 @@ cudaError_t launch_d(const Shape& s, const HostRange& r, const void* q, const vo
   p.Hkv = s.Hkv;
   p.G = s.Hq / s.Hkv;
   p.n_ctas_per_host = ((s.n + kRows - 1) / kRows + 1) / 2;
-  p.hb = r.hb;
-  p.he = r.he;
+  p.h0 = r.h0;
+  p.hcount = r.count;
+  p.hstride = r.stride;
   p.q_row0 = r.q_row0;
   p.k_row0 = r.k_row0;
   p.anchor_row0 = r.anchor_row0;
@@ -512,7 +515,7 @@ cudaError_t launch_d(const Shape& s, const HostRange& r, const void* q, const vo
   cudaError_t e = cudaFuncSetAttribute(apb_attention_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_ctas_per_host, s.Hq, r.he - r.hb);
+  dim3 grid(p.n_ctas_per_host, s.Hq, r.count);
   apb_attention_kernel<D><<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, mPK, mPV, p);
   return cudaGetLastError();
 }

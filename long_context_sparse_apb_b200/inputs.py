@@ -204,15 +204,17 @@ def generate(cfg: APBConfig) -> Dict[str, torch.Tensor]:
     return out
 
 
-def generate_local(cfg: APBConfig, host_begin: int, host_end: int) -> Dict[str, torch.Tensor]:
-    """What one GPU of a host-sharded prefill holds: q of hosts
-    [host_begin, host_end) and k/v with the anchor's rows [0, A) first, then
-    those hosts' rows (each host prepends the anchor to its block).  Values
-    equal the matching rows of generate(cfg)."""
+def generate_local(cfg: APBConfig, host_begin: int, host_end: int,
+                   host_stride: int = 1) -> Dict[str, torch.Tensor]:
+    """What one GPU of a host-sharded prefill holds: q of the hosts
+    range(host_begin, host_end, host_stride) and k/v with the anchor's rows
+    [0, A) first, then those hosts' rows, in that order (each host prepends
+    the anchor to its block).  Values equal the matching rows of
+    generate(cfg)."""
     n, A = cfg.block_len, cfg.anchor_len
     q0 = _q_block(cfg, 0)
     qseg_mean = _qseg_mean(cfg, q0)
-    hosts = range(host_begin, host_end)
+    hosts = range(host_begin, host_end, host_stride)
     q = torch.cat([(q0 if h == 0 else _q_block(cfg, h)).to(torch.bfloat16) for h in hosts])
     out = {"q": q}
     for name, tid in (("k", _TID_K), ("v", _TID_V)):

@@ -4,23 +4,26 @@ each host prepends the anchor block to its context block, compresses its KV
 with the retaining heads, the compressed blocks are all-gathered, and each host
 attends over anchor + passing block + its own block).
 
-One process per GPU; rank r owns the contiguous hosts [r*H/W, (r+1)*H/W).
-Per step, on each rank:
+One process per GPU.  Rank r of W owns H/W hosts, either round-robin (hosts
+r, r+W, r+2W, ...: the default, which balances the work, since a host's
+attention grows with its index through the passing block) or contiguous
+(hosts [r*H/W, (r+1)*H/W)).  Per step, on each rank:
   1. for every owned host: score + top-k (apb_score_compress on that host's
      block) and its compressed block, written straight into the host's rows
      [h*keep, (h+1)*keep) of a full token-major passing buffer
      (apb_build_passing);
-  2. one all-gather of the passing buffer's K rows and one of its V rows
-     (each rank contributes its contiguous chunk; the result is all hosts'
-     blocks in host order, because ranks own hosts in order);
+  2. all-gathers of the passing buffer's K and V rows that leave every
+     host's block in host order: round-robin, one per round i over the rows
+     of hosts [i*W, (i+1)*W) (rank r contributes host i*W + r); contiguous,
+     one over the whole buffer (rank r contributes its hosts' chunk);
   3. attention of the owned hosts on the rank-local buffers
-     (apb_block_attention_hosts).
+     (apb_block_attention_host_set).
 Every step of the data path runs in the library's kernels; the exchange is
 the collective passed in (NCCL all_gather_into_tensor between GPUs).
 """
 from __future__ import annotations
 
-from typing import Callable, Optional, Tuple
+from typing import Callable, List, Optional, Tuple
 
 import torch
 
@@ -33,6 +36,31 @@ def host_range(n_hosts: int, rank: int, world: int) -> Tuple[int, int]:
         raise ValueError(f"{n_hosts} hosts do not split evenly over {world} ranks")
     per = n_hosts // world
     return rank * per, (rank + 1) * per
+
+
+def host_set(n_hosts: int, rank: int, world: int, order: str = "round_robin") -> Tuple[int, int, int]:
+    """(first, count, stride) of the hosts owned by `rank`: round_robin owns
+    rank, rank+W, ...; contiguous owns [rank*H/W, (rank+1)*H/W)."""
+    first, end = host_range(n_hosts, rank, world)
+    if order == "contiguous":
+        return first, end - first, 1
+    if order == "round_robin":
+        return rank, end - first, world
+    raise ValueError(f"unknown host order {order!r}")
+
+
+def exchange_chunks(n_hosts: int, keep: int, rank: int, world: int,
+                    order: str = "round_robin") -> List[Tuple[slice, slice]]:
+    """Row ranges (full, chunk) of the passing buffer for the all-gathers of
+    the exchange: after all_gather(full, chunk) for each pair (every rank
+    passing its own chunk, which lies inside full at position `rank`), the
+    buffer holds every host's block in host order."""
+    first, count, stride = host_set(n_hosts, rank, world, order)
+    if order == "contiguous":
+        return [(slice(0, n_hosts * keep), slice(first * keep, (first + count) * keep))]
+    W = world
+    return [(slice(i * W * keep, (i + 1) * W * keep),
+             slice((i * W + rank) * keep, (i * W + rank + 1) * keep)) for i in range(count)]
 
 
 def kv_head_range(n_kv_heads: int, rank: int, world: int) -> Tuple[int, int]:
@@ -87,10 +115,12 @@ class ShardedPrefill:
     """
 
     def __init__(self, c: apb.Config, rank: int, world: int, device="cuda",
-                 all_gather: Optional[Callable] = None):
+                 all_gather: Optional[Callable] = None, order: str = "round_robin"):
         self.c = c
         self.rank, self.world = rank, world
-        self.hb, self.he = host_range(c.n_hosts, rank, world)
+        self.order = order
+        self.first, self.count, self.stride = host_set(c.n_hosts, rank, world, order)
+        self.hosts = [self.first + i * self.stride for i in range(self.count)]
         self.all_gather = all_gather
         n, keep, hkv, d = c.block_len, c.keep, c.n_kv_heads, c.head_dim
         # single-host config for the per-host compression calls
@@ -100,17 +130,17 @@ class ShardedPrefill:
                                   softmax_scale=c.softmax_scale)
         dev = torch.device(device)
         self.workspace = apb.new_workspace(self.c1, dev)
-        self.idx = torch.empty((self.he - self.hb, 1, hkv, keep), dtype=torch.int32, device=dev)
+        self.idx = torch.empty((self.count, 1, hkv, keep), dtype=torch.int32, device=dev)
         shape = (c.n_hosts * keep, hkv, d)
         self.pass_k = torch.empty(shape, dtype=torch.bfloat16, device=dev)
         self.pass_v = torch.empty(shape, dtype=torch.bfloat16, device=dev)
-        self.out = torch.empty(((self.he - self.hb) * n, c.n_q_heads, d), dtype=torch.bfloat16,
+        self.out = torch.empty((self.count * n, c.n_q_heads, d), dtype=torch.bfloat16,
                                device=dev)
 
     def compress(self, q, kv_k, kv_v, w1, b1, w2, b2, stream=None, query_aware=False):
         """Steps 1: compressed blocks of the owned hosts into their rows."""
         n, A, keep = self.c.block_len, self.c.anchor_len, self.c.keep
-        for i, h in enumerate(range(self.hb, self.he)):
+        for i, h in enumerate(self.hosts):
             qs = q[i * n:(i + 1) * n]
             ks = kv_k[A + i * n:A + (i + 1) * n]
             vs = kv_v[A + i * n:A + (i + 1) * n]
@@ -126,15 +156,16 @@ class ShardedPrefill:
         keep = self.c.keep
         if self.all_gather is None or keep == 0 or self.world == 1:
             return
-        rows = slice(self.hb * keep, self.he * keep)
-        self.all_gather(self.pass_k, self.pass_k[rows])
-        self.all_gather(self.pass_v, self.pass_v[rows])
+        for full, chunk in exchange_chunks(self.c.n_hosts, keep, self.rank, self.world,
+                                           self.order):
+            self.all_gather(self.pass_k[full], self.pass_k[chunk])
+            self.all_gather(self.pass_v[full], self.pass_v[chunk])
 
     def attend(self, q, kv_k, kv_v, stream=None, lse=None):
         """Step 3: attention of the owned hosts."""
-        out, _ = apb.block_attention_hosts(self.c, self.hb, self.he, q, kv_k, kv_v, self.pass_k,
-                                           self.pass_v, out=self.out, lse=lse,
-                                           workspace=self.workspace, stream=stream)
+        out, _ = apb.block_attention_host_set(self.c, self.first, self.count, self.stride, q, kv_k,
+                                              kv_v, self.pass_k, self.pass_v, out=self.out,
+                                              lse=lse, workspace=self.workspace, stream=stream)
         return out
 
     def __call__(self, q, kv_k, kv_v, w1, b1, w2, b2, stream=None):

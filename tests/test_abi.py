@@ -123,6 +123,12 @@ def test_host_range_and_query_aware_checks():
     st = apb._lib.apb_block_attention_hosts(ctypes.byref(c), 1, 3, None, *([FAKE] * 5), None,
                                             FAKE, 256, None)
     assert st == apb.APB_ERR_INVALID_ARG                  # q is NULL
+    # strided host sets (TINY has 4 hosts): the last host must exist, count and
+    # stride must be positive
+    for first, count, stride in ((0, 0, 1), (0, 2, 0), (-1, 2, 1), (1, 2, 3), (0, 5, 1),
+                                 (3, 2, 1)):
+        assert apb._lib.apb_block_attention_host_set(ctypes.byref(c), first, count, stride,
+                                                     *args) == apb.APB_ERR_INVALID_ARG
     # the query-aware variant needs room for its bias next to the weight split
     st = apb._lib.apb_score_compress_query_aware(ctypes.byref(c), *([FAKE] * 8), FAKE, FAKE,
                                                  256 + 2 * 256 * 192 * 4, None)

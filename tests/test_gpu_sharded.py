@@ -11,16 +11,17 @@ from long_context_sparse_apb_b200 import inputs
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("order", ["round_robin", "contiguous"])
 @pytest.mark.parametrize("cfg,world", [
     (inputs.TINY, 2), (inputs.TINY, 4),
     (inputs.TINY.replace(n_hosts=6, block_len=300, anchor_len=75, keep=50, n_q_heads=8,
                          head_dim=128, seed=21), 3),
 ], ids=["tiny_w2", "tiny_w4", "ragged_w3"])
-def test_sharded_equals_single_gpu(cfg, world):
+def test_sharded_equals_single_gpu(cfg, world, order):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from long_context_sparse_apb_b200 import _lib as apb
-    from long_context_sparse_apb_b200.sharded import ShardedPrefill
+    from long_context_sparse_apb_b200.sharded import ShardedPrefill, exchange_chunks
 
     x = inputs.generate(cfg)
     c = apb.make_config(cfg)
@@ -29,23 +30,26 @@ def test_sharded_equals_single_gpu(cfg, world):
 
     ranks, locs = [], []
     for r in range(world):
-        sp = ShardedPrefill(c, r, world)
-        loc = {k: v.cuda() for k, v in inputs.generate_local(cfg, sp.hb, sp.he).items()}
+        sp = ShardedPrefill(c, r, world, order=order)
+        loc = {k: v.cuda() for k, v in inputs.generate_local(
+            cfg, sp.first, sp.first + sp.count * sp.stride, sp.stride).items()}
         sp.compress(loc["q"], loc["k"], loc["v"], loc["w1"], loc["b1"], loc["w2"], loc["b2"])
         ranks.append(sp)
         locs.append(loc)
     keep = cfg.keep
-    for src in ranks:                       # the all-gather, emulated
-        rows = slice(src.hb * keep, src.he * keep)
-        for dst in ranks:
-            if dst is not src:
-                dst.pass_k[rows].copy_(src.pass_k[rows])
-                dst.pass_v[rows].copy_(src.pass_v[rows])
-    outs = [sp.attend(loc["q"], loc["k"], loc["v"]) for sp, loc in zip(ranks, locs)]
-    torch.cuda.synchronize()
-    for sp in ranks:
+    for r, src in enumerate(ranks):         # the all-gathers, emulated
+        for _, rows in exchange_chunks(cfg.n_hosts, keep, r, world, order):
+            for dst in ranks:
+                if dst is not src:
+                    dst.pass_k[rows].copy_(src.pass_k[rows])
+                    dst.pass_v[rows].copy_(src.pass_v[rows])
+    n = cfg.block_len
+    for sp, loc in zip(ranks, locs):
+        out = sp.attend(loc["q"], loc["k"], loc["v"])
+        torch.cuda.synchronize()
         assert apb.device_status(sp.workspace) == apb.APB_OK
-    assert torch.equal(torch.cat(outs), ref)
+        for i, h in enumerate(sp.hosts):
+            assert torch.equal(out[i * n:(i + 1) * n], ref[h * n:(h + 1) * n]), (order, h)
 
 
 @pytest.mark.parametrize("world", [2])

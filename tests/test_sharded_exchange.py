@@ -1,13 +1,13 @@
 """The all-gather of the host-sharded prefill on CPU ranks (gloo, world
 size 2): every rank ends with all ranks' compressed-block rows in host order,
-and the host ranges partition the hosts."""
+for both host assignments, and the host sets partition the hosts."""
 import os
 import socket
 
 import pytest
 import torch.multiprocessing as mp
 
-from long_context_sparse_apb_b200.sharded import host_range
+from long_context_sparse_apb_b200.sharded import exchange_chunks, host_range, host_set
 
 
 def test_host_ranges_partition():
@@ -19,6 +19,30 @@ def test_host_ranges_partition():
         host_range(8, 0, 3)
 
 
+@pytest.mark.parametrize("order", ["round_robin", "contiguous"])
+def test_host_sets_partition_and_chunks_tile_the_buffer(order):
+    for H, W, keep in ((8, 1, 3), (8, 2, 3), (8, 4, 2), (8, 8, 1), (16, 4, 5)):
+        owned = []
+        for r in range(W):
+            first, count, stride = host_set(H, r, W, order)
+            owned += [first + i * stride for i in range(count)]
+            for full, chunk in exchange_chunks(H, keep, r, W, order):
+                # each rank's chunk is its slot `r` of an all-gather over `full`
+                assert full.stop - full.start == W * (chunk.stop - chunk.start)
+                assert chunk.start - full.start == r * (chunk.stop - chunk.start)
+                hosts = range(chunk.start // keep, chunk.stop // keep)
+                assert all((h - first) % stride == 0 and 0 <= (h - first) // stride < count
+                           for h in hosts)          # a rank sends only its own hosts' rows
+        assert sorted(owned) == list(range(H))
+    # round-robin balances work that grows linearly with the host index
+    def spread(order, H=8, W=2):
+        loads = []
+        for r in range(W):
+            first, count, stride = host_set(H, r, W, order)
+            loads.append(sum(1 + first + i * stride for i in range(count)))
+        return max(loads) - min(loads)
+    assert spread("round_robin") < spread("contiguous")
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -27,30 +51,32 @@ def _free_port():
     return p
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, order):
     os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
                       MASTER_PORT=str(port))
     import torch
     import torch.distributed as dist
-    from long_context_sparse_apb_b200.sharded import host_range, list_all_gather
+    from long_context_sparse_apb_b200.sharded import exchange_chunks, host_set, list_all_gather
 
     dist.init_process_group("gloo")
     H, keep, hkv, d = 4, 3, 2, 4
     full = torch.zeros(H * keep, hkv, d)
-    hb, he = host_range(H, rank, world)
-    for h in range(hb, he):                 # this rank's compressed blocks
+    first, count, stride = host_set(H, rank, world, order)
+    for h in range(first, first + count * stride, stride):     # this rank's blocks
         full[h * keep:(h + 1) * keep] = 100 * h + torch.arange(keep * hkv * d).reshape(keep, hkv, d)
-    list_all_gather()(full, full[hb * keep:he * keep])
+    for rows, chunk in exchange_chunks(H, keep, rank, world, order):
+        list_all_gather()(full[rows], full[chunk])
     q.put((rank, full.numpy()))
     dist.destroy_process_group()
 
 
-def test_exchange_two_gloo_ranks():
+@pytest.mark.parametrize("order", ["round_robin", "contiguous"])
+def test_exchange_two_gloo_ranks(order):
     import torch
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q, order)) for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
