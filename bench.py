@@ -319,15 +319,16 @@ def run_gpu(args, cfg):
     value = world * cfg.seq_len / (max_ms / 1e3 / args.steps)
 
     # ---- end to end through the public API with pinned host buffers: every
-    # step copies its inputs in and its output back; PrefillPipeline overlaps
-    # one step's copies with another step's compute
+    # step copies its inputs in and its output back; StreamedPrefill streams
+    # each step host by host, so its copies overlap its own compute and the
+    # other step's
     hx = {k: v.pin_memory() for k, v in x.items() if k != "needles"}
     hout = [torch.empty(run.out.shape, dtype=run.out.dtype).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in hx.values())
     d2h = hout[0].numel() * hout[0].element_size()
     del run, xd, pws, pout
     torch.cuda.empty_cache()
-    pipe = apb.PrefillPipeline(c, device=dev, depth=2)
+    pipe = apb.StreamedPrefill(c, device=dev, depth=2)
     for i in range(max(2, args.warmup)):
         pipe.submit(hx, hout[i % 2])
     pipe.synchronize()
@@ -340,13 +341,16 @@ def run_gpu(args, cfg):
     e0.record(pipe.h2d)
     for i in range(e2e_steps):
         pipe.submit(hx, hout[i % 2])
-    pipe.d2h.wait_stream(pipe.comp)
+    for s in [pipe.comp] + pipe.att:
+        pipe.d2h.wait_stream(s)
     e1.record(pipe.d2h)
     pipe.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     wall_ms = (time.perf_counter() - t0) * 1e3
     barrier(world)
     e2e_value = world * cfg.seq_len / (e2e_ms / 1e3 / e2e_steps)
+    if any(apb.device_status(w) != apb.APB_OK for w in pipe.workspaces()):
+        raise RuntimeError("device status not OK after the end-to-end steps")
     del pipe
     torch.cuda.empty_cache()
     xd = {k: v.to(dev) for k, v in x.items() if k != "needles"}
@@ -402,9 +406,10 @@ def run_gpu(args, cfg):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms": e2e_ms,
                 "host_wall_ms": wall_ms,
-                "how": "PrefillPipeline: pinned H2D copies, one apb_prefill call and the D2H copy of "
-                       "the output on three streams, two slots, copies of one step overlapping "
-                       "another step's compute"},
+                "how": "StreamedPrefill: pinned host buffers; per step the H2D copies, the "
+                       "compression, the attention (two streams) and the D2H copies run host by "
+                       "host on their own streams, two slots; copy-in of host h+1 overlaps host "
+                       "h's compute, and host h's output goes back as soon as it is attended"},
         "gpu_launches": args.steps * (5 if cfg.keep > 0 and cfg.n_hosts > 1 else 1),
         "clocks": clk,
     }

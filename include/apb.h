@@ -154,6 +154,19 @@ apb_status apb_block_attention(const apb_config* cfg, const void* q, const void*
                                void* out, float* lse, void* workspace, size_t ws_bytes,
                                void* stream);
 
+/* Step 3 for the hosts [host_begin, host_end) only, on the whole-sequence
+ * buffers of apb_block_attention (q, k, v, out [N, ...]; lse [Hq, N]): the
+ * rows of those hosts in out (and lse) are written, nothing else.  Lets a
+ * caller attend host h as soon as its own rows and the compressed blocks of
+ * hosts 0..h-1 are in place (main features: each host attends over the
+ * anchor, the passing block of the hosts before it and its own block), e.g.
+ * while later hosts' inputs are still being copied in.
+ * 0 <= host_begin < host_end <= n_hosts, else APB_ERR_INVALID_ARG. */
+apb_status apb_block_attention_range(const apb_config* cfg, int32_t host_begin, int32_t host_end,
+                                     const void* q, const void* k, const void* v,
+                                     const void* pass_k, const void* pass_v, void* out,
+                                     float* lse, void* workspace, size_t ws_bytes, void* stream);
+
 /* Step 3 for a range of hosts on rank-local buffers (main features: the
  * sequence is split over hosts, each host's context block is preceded by the
  * anchor block, and the passing block is built from the all-gathered

@@ -52,6 +52,8 @@ _lib.apb_block_attention.restype = ctypes.c_int
 _lib.apb_block_attention_hosts.argtypes = ([ctypes.POINTER(Config), ctypes.c_int32, ctypes.c_int32]
                                            + [_P] * 8 + [ctypes.c_size_t, _P])
 _lib.apb_block_attention_hosts.restype = ctypes.c_int
+_lib.apb_block_attention_range.argtypes = _lib.apb_block_attention_hosts.argtypes
+_lib.apb_block_attention_range.restype = ctypes.c_int
 _lib.apb_block_attention_host_set.argtypes = ([ctypes.POINTER(Config)] + [ctypes.c_int32] * 3
                                               + [_P] * 8 + [ctypes.c_size_t, _P])
 _lib.apb_block_attention_host_set.restype = ctypes.c_int
@@ -239,6 +241,33 @@ def block_attention(c: Config, q, k, v, pass_k, pass_v, out=None, lse=None, want
                                   _ptr(pass_v) if use_pass else None, _ptr(out), _ptr(lse),
                                   _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "apb_block_attention")
+    return out, lse
+
+
+def block_attention_range(c: Config, host_begin: int, host_end: int, q, k, v, pass_k, pass_v,
+                          out, lse=None, workspace=None, stream=None):
+    """apb_block_attention_range: attention of hosts [host_begin, host_end)
+    on the whole-sequence buffers; writes only those hosts' rows of out (and
+    lse).  Returns (out, lse)."""
+    N, hq, hkv, d = _dims(c)
+    _want(q, "q", torch.bfloat16, (N, hq, d))
+    _want(k, "k", torch.bfloat16, (N, hkv, d))
+    _want(v, "v", torch.bfloat16, (N, hkv, d))
+    _want(out, "out", torch.bfloat16, (N, hq, d))
+    use_pass = c.keep > 0 and host_end > 1
+    if use_pass:
+        shape = (c.n_hosts * c.keep, hkv, d)
+        _want(pass_k, "pass_k", torch.bfloat16, shape)
+        _want(pass_v, "pass_v", torch.bfloat16, shape)
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (hq, N))
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    st = _lib.apb_block_attention_range(ctypes.byref(c), host_begin, host_end, _ptr(q), _ptr(k),
+                                        _ptr(v), _ptr(pass_k) if use_pass else None,
+                                        _ptr(pass_v) if use_pass else None, _ptr(out), _ptr(lse),
+                                        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "apb_block_attention_range")
     return out, lse
 
 
@@ -445,4 +474,125 @@ class PrefillPipeline:
 
     def synchronize(self) -> None:
         for st in (self.h2d, self.comp, self.d2h):
+            st.synchronize()
+
+
+class StreamedPrefill:
+    """Prefills of successive sequences from pinned host memory, streamed host
+    by host: host h's rows are copied in, compressed and attended while the
+    rows of later hosts are still on their way, and its output rows go back as
+    soon as they are done.  So a step's copies overlap its own compute, not
+    only another step's, and the first copy-in and last copy-out of a run
+    cost one host's rows instead of a whole sequence.
+
+    Per step (streams ordered by events): the H2D stream copies the weights,
+    then host 0, 1, ... (q, k, v rows); one compute stream compresses host h
+    (apb_score_compress and apb_build_passing on host h's rows with a
+    one-host config, writing rows [h*keep, (h+1)*keep) of the passing
+    buffers) once its rows are in; two attention streams take hosts in turn
+    (apb_block_attention_range for host h once its rows and the compressed
+    blocks of hosts 0..h-1 are in place), so one host's launch fills the
+    tail of the other's; the D2H stream copies host h's output rows out.
+    The last host's compression is skipped (no host follows it).  `depth`
+    slots own the device buffers; a slot is reused only after all its work,
+    including the copy-out, has finished.  synchronize() waits for
+    everything queued."""
+
+    def __init__(self, c: Config, device="cuda", depth: int = 2):
+        N, hq, hkv, d = _dims(c)
+        dev = torch.device(device)
+        self.c = c
+        self.depth = depth
+        self.H, self.n = c.n_hosts, c.block_len
+        self.c1 = make_config(None, n_hosts=1, block_len=c.block_len, anchor_len=c.anchor_len,
+                              query_len=c.query_len, keep=c.keep, n_q_heads=c.n_q_heads,
+                              n_kv_heads=c.n_kv_heads, head_dim=c.head_dim,
+                              mlp_hidden=c.mlp_hidden, softmax_scale=c.softmax_scale)
+        self.h2d = torch.cuda.Stream(dev)
+        self.comp = torch.cuda.Stream(dev)
+        self.att = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+        self.d2h = torch.cuda.Stream(dev)
+        self.slots = []
+        for _ in range(depth):
+            x = {"q": torch.empty((N, hq, d), dtype=torch.bfloat16, device=dev),
+                 "k": torch.empty((N, hkv, d), dtype=torch.bfloat16, device=dev),
+                 "v": torch.empty((N, hkv, d), dtype=torch.bfloat16, device=dev),
+                 "w1": torch.empty((hkv, c.mlp_hidden, 3 * d), dtype=torch.float32, device=dev),
+                 "b1": torch.empty((hkv, c.mlp_hidden), dtype=torch.float32, device=dev),
+                 "w2": torch.empty((hkv, c.mlp_hidden), dtype=torch.float32, device=dev),
+                 "b2": torch.empty((hkv,), dtype=torch.float32, device=dev)}
+            shape = (max(self.H, 1) * c.keep, hkv, d)
+            self.slots.append({
+                "x": x, "used": False,
+                "out": torch.empty((N, hq, d), dtype=torch.bfloat16, device=dev),
+                "idx": torch.empty((self.H, 1, hkv, c.keep), dtype=torch.int32, device=dev),
+                "pass_k": torch.empty(shape, dtype=torch.bfloat16, device=dev),
+                "pass_v": torch.empty(shape, dtype=torch.bfloat16, device=dev),
+                "ws_comp": new_workspace(self.c1, dev),
+                "ws_att": [torch.zeros(256, dtype=torch.uint8, device=dev) for _ in range(2)],
+                "ev_in": [torch.cuda.Event() for _ in range(self.H)],
+                "ev_pass": [torch.cuda.Event() for _ in range(self.H)],
+                "ev_att": [torch.cuda.Event() for _ in range(self.H)],
+                "ev_done": [torch.cuda.Event() for _ in range(4)],   # comp, att0, att1, d2h
+            })
+        self.i = 0
+
+    def workspaces(self):
+        """Every workspace (for apb_device_status)."""
+        return [w for sl in self.slots for w in [sl["ws_comp"]] + sl["ws_att"]]
+
+    def submit(self, host: dict, host_out: torch.Tensor) -> None:
+        """host: pinned CPU tensors q, k, v, w1, b1, w2, b2; host_out: pinned
+        CPU bf16 [N, Hq, d] receiving this step's output."""
+        sl = self.slots[self.i % self.depth]
+        self.i += 1
+        H, n, keep = self.H, self.n, self.c.keep
+        x = sl["x"]
+        compress = keep > 0 and H > 1
+        with torch.cuda.stream(self.h2d):
+            if sl["used"]:
+                for e in sl["ev_done"]:              # the slot's previous step is over
+                    self.h2d.wait_event(e)
+            for name in ("w1", "b1", "w2", "b2"):
+                x[name].copy_(host[name], non_blocking=True)
+            for h in range(H):
+                rows = slice(h * n, (h + 1) * n)
+                for name in ("q", "k", "v"):
+                    x[name][rows].copy_(host[name][rows], non_blocking=True)
+                sl["ev_in"][h].record(self.h2d)
+        with torch.cuda.stream(self.comp):
+            if compress:
+                for h in range(H - 1):
+                    rows = slice(h * n, (h + 1) * n)
+                    self.comp.wait_event(sl["ev_in"][h])
+                    score_compress(self.c1, x["q"][rows], x["k"][rows], x["v"][rows], x["w1"],
+                                   x["b1"], x["w2"], x["b2"], idx=sl["idx"][h],
+                                   workspace=sl["ws_comp"], stream=self.comp)
+                    build_passing(self.c1, x["k"][rows], x["v"][rows], sl["idx"][h],
+                                  sl["pass_k"][h * keep:(h + 1) * keep],
+                                  sl["pass_v"][h * keep:(h + 1) * keep], stream=self.comp)
+                    sl["ev_pass"][h].record(self.comp)
+            sl["ev_done"][0].record(self.comp)
+        for h in range(H):
+            s = self.att[h % 2]
+            with torch.cuda.stream(s):
+                s.wait_event(sl["ev_in"][h])
+                if compress and h >= 1:
+                    s.wait_event(sl["ev_pass"][h - 1])
+                block_attention_range(self.c, h, h + 1, x["q"], x["k"], x["v"], sl["pass_k"],
+                                      sl["pass_v"], sl["out"], workspace=sl["ws_att"][h % 2],
+                                      stream=s)
+                sl["ev_att"][h].record(s)
+        for j, s in enumerate(self.att):
+            sl["ev_done"][1 + j].record(s)
+        with torch.cuda.stream(self.d2h):
+            for h in range(H):
+                rows = slice(h * n, (h + 1) * n)
+                self.d2h.wait_event(sl["ev_att"][h])
+                host_out[rows].copy_(sl["out"][rows], non_blocking=True)
+            sl["ev_done"][3].record(self.d2h)
+        sl["used"] = True
+
+    def synchronize(self) -> None:
+        for st in [self.h2d, self.comp, self.d2h] + self.att:
             st.synchronize()

@@ -235,6 +235,14 @@ apb_status apb_block_attention_hosts(const apb_config* cfg, int32_t host_begin, 
                         stream);
 }
 
+apb_status apb_block_attention_range(const apb_config* cfg, int32_t host_begin, int32_t host_end,
+                                     const void* q, const void* k, const void* v,
+                                     const void* pass_k, const void* pass_v, void* out,
+                                     float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return attention_impl("apb_block_attention_range", cfg, host_begin, host_end - host_begin, 1,
+                        false, q, k, v, pass_k, pass_v, out, lse, workspace, ws_bytes, stream);
+}
+
 apb_status apb_block_attention_host_set(const apb_config* cfg, int32_t host_first,
                                         int32_t host_count, int32_t host_stride, const void* q,
                                         const void* kv_k, const void* kv_v, const void* pass_k,

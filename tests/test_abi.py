@@ -123,6 +123,9 @@ def test_host_range_and_query_aware_checks():
     st = apb._lib.apb_block_attention_hosts(ctypes.byref(c), 1, 3, None, *([FAKE] * 5), None,
                                             FAKE, 256, None)
     assert st == apb.APB_ERR_INVALID_ARG                  # q is NULL
+    for hb, he in ((0, 0), (2, 1), (-1, 2), (0, 5)):
+        assert apb._lib.apb_block_attention_range(ctypes.byref(c), hb, he, *args) == \
+            apb.APB_ERR_INVALID_ARG
     # strided host sets (TINY has 4 hosts): the last host must exist, count and
     # stride must be positive
     for first, count, stride in ((0, 0, 1), (0, 2, 0), (-1, 2, 1), (1, 2, 3), (0, 5, 1),

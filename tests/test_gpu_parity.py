@@ -157,6 +157,38 @@ def test_pipeline_matches_direct_calls(apb):
 
 
 @pytest.mark.parametrize("cfg", [inputs.TINY,
+                                 inputs.TINY.replace(n_hosts=5, block_len=300, anchor_len=75,
+                                                     keep=40, n_q_heads=8, head_dim=128, seed=14),
+                                 inputs.TINY.replace(n_hosts=1, seed=15)],
+                         ids=["tiny", "ragged_5_hosts", "one_host"])
+def test_streamed_prefill_matches_direct_calls(apb, cfg):
+    # StreamedPrefill (host-by-host copies, compression and attention on
+    # several streams) returns, for each submitted step, exactly what the
+    # three direct calls return
+    cfgs = [cfg, cfg.replace(seed=cfg.seed + 100)]
+    xs = [inputs.generate(k) for k in cfgs]
+    c = apb.make_config(cfg)
+    direct = []
+    for x in xs:
+        xd = _to_dev(x)
+        run = apb.Prefill(c)
+        direct.append(run(xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"], xd["b2"]).cpu())
+    pipe = apb.StreamedPrefill(c, depth=2)
+    outs = []
+    for step in range(5):
+        x = xs[step % 2]
+        hx = {k: v.pin_memory() for k, v in x.items() if k != "needles"}
+        ho = torch.empty_like(direct[0]).pin_memory()
+        pipe.submit(hx, ho)
+        outs.append((step % 2, ho, hx))
+    pipe.synchronize()
+    for ws in pipe.workspaces():
+        assert apb.device_status(ws) == apb.APB_OK
+    for which, ho, _ in outs:
+        assert torch.equal(ho, direct[which])
+
+
+@pytest.mark.parametrize("cfg", [inputs.TINY,
                                  inputs.TINY.replace(n_hosts=3, block_len=300, anchor_len=75,
                                                      query_len=0, keep=40, seed=9),
                                  inputs.TINY.replace(n_q_heads=10, n_kv_heads=2, head_dim=128,
