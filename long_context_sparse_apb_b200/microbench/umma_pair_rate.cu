@@ -1,5 +1,5 @@
 // Sustained tcgen05.mma.cta_group::2 rate (M = 256 split over the two SMs of
-// a cluster pair; the leader issues, a multicast commit signals both CTAs) for
+// a cluster pair; the leader issues, one commit to each CTA's barrier) for
 // SS 256x128x16, SS 256x256x16 and TS 256x128x16, to compare the per-SM rate
 // of paired MMAs with the single-SM shapes of umma_rate.cu.
 #include <cstdio>
@@ -50,16 +50,31 @@ umma2_rate(int mode, int iters, long long* out, unsigned* err) {
     const uint64_t dA = ptx::sdesc_sw128(ptx::smem_u32(sm), 16, 1024);
     const uint64_t dB = ptx::sdesc_sw128(ptx::smem_u32(sm + 16384), 16, 1024);
     long long t0 = clock64();
-    for (int it = 0; it < iters; ++it) {
+    // straight-line UMMA runs (no branch between consecutive UMMAs)
+    if (mode == 2) {
+      for (int it = 0; it < iters; ++it) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk & 3) * 32) >> 4;
-        if (mode == 2) umma2_ts(tmem, tmem + 256 + kk * 8, dB + off, idesc, 1u);
-        else umma2_ss(tmem, dA + off, dB + off, idesc, 1u);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk & 3) * 32) >> 4;
+          umma2_ts(tmem, tmem + 256 + kk * 8, dB + off, idesc, 1u);
+        }
+      }
+    } else {
+      for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk & 3) * 32) >> 4;
+          umma2_ss(tmem, dA + off, dB + off, idesc, 1u);
+        }
       }
     }
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-                 :: "r"(ptx::smem_u32(&bar)), "h"((unsigned short)3) : "memory");
+    // one arrival on each CTA's barrier once every UMMA above has completed
+    uint32_t peer_bar;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 1;" : "=r"(peer_bar) : "r"(ptx::smem_u32(&bar)));
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(ptx::smem_u32(&bar)) : "memory");
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(peer_bar) : "memory");
     out[blockIdx.x] = clock64() - t0;   // issue time only; completion below
   }
   if (threadIdx.x == 0) {

@@ -31,14 +31,24 @@ __global__ void __launch_bounds__(128, 1) umma_rate(int mode, int iters, long lo
     const uint64_t dA = ptx::sdesc_sw128(ptx::smem_u32(sm), 16, 1024);
     const uint64_t dB = ptx::sdesc_sw128(ptx::smem_u32(sm + 16384), 16, 1024);
     long long t0 = clock64();
-    for (int it = 0; it < iters; ++it) {
+    // one straight-line run of UMMAs per mode: a branch between consecutive
+    // UMMAs (e.g. choosing the form inside the unrolled loop) slows the
+    // stream to ~104 (SS) / ~93 (TS) cycles per 128x128x16 UMMA
+    if (mode == 2) {
+      for (int it = 0; it < iters; ++it) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk & 3) * 32) >> 4;   // stay inside the first 64-column block
-        if (mode == 2)
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk & 3) * 32) >> 4;   // stay inside the first 64-column block
           ptx::umma_bf16_ts(tmem, tmem + 256 + kk * 8, dB + off, idesc, 1u);
-        else
+        }
+      }
+    } else {
+      for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk & 3) * 32) >> 4;
           ptx::umma_bf16_ss(tmem, dA + off, dB + off, idesc, 1u);
+        }
       }
     }
     ptx::umma_commit(&bar);
