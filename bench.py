@@ -328,7 +328,10 @@ def run_gpu(args, cfg):
     d2h = hout[0].numel() * hout[0].element_size()
     del run, xd, pws, pout
     torch.cuda.empty_cache()
-    pipe = apb.StreamedPrefill(c, device=dev, depth=2)
+    # host-by-host streaming pays per-host launches; for short blocks the
+    # whole-step pipeline (one apb_prefill per step) is the faster public path
+    streamed = cfg.block_len >= 4096
+    pipe = (apb.StreamedPrefill if streamed else apb.PrefillPipeline)(c, device=dev, depth=2)
     for i in range(max(2, args.warmup)):
         pipe.submit(hx, hout[i % 2])
     pipe.synchronize()
@@ -341,7 +344,7 @@ def run_gpu(args, cfg):
     e0.record(pipe.h2d)
     for i in range(e2e_steps):
         pipe.submit(hx, hout[i % 2])
-    for s in [pipe.comp] + pipe.att:
+    for s in [pipe.comp] + (pipe.att if streamed else []):
         pipe.d2h.wait_stream(s)
     e1.record(pipe.d2h)
     pipe.synchronize()
@@ -349,7 +352,8 @@ def run_gpu(args, cfg):
     wall_ms = (time.perf_counter() - t0) * 1e3
     barrier(world)
     e2e_value = world * cfg.seq_len / (e2e_ms / 1e3 / e2e_steps)
-    if any(apb.device_status(w) != apb.APB_OK for w in pipe.workspaces()):
+    wss = pipe.workspaces() if streamed else [sl["ws"] for sl in pipe.slots]
+    if any(apb.device_status(w) != apb.APB_OK for w in wss):
         raise RuntimeError("device status not OK after the end-to-end steps")
     del pipe
     torch.cuda.empty_cache()
@@ -406,10 +410,14 @@ def run_gpu(args, cfg):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms": e2e_ms,
                 "host_wall_ms": wall_ms,
-                "how": "StreamedPrefill: pinned host buffers; per step the H2D copies, the "
-                       "compression, the attention (two streams) and the D2H copies run host by "
-                       "host on their own streams, two slots; copy-in of host h+1 overlaps host "
-                       "h's compute, and host h's output goes back as soon as it is attended"},
+                "how": ("StreamedPrefill: pinned host buffers; per step the H2D copies, the "
+                        "compression, the attention (two streams) and the D2H copies run host by "
+                        "host on their own streams, two slots; copy-in of host h+1 overlaps host "
+                        "h's compute, and host h's output goes back as soon as it is attended"
+                        if streamed else
+                        "PrefillPipeline (blocks shorter than 4096 rows): pinned H2D copies, one "
+                        "apb_prefill call and the D2H copy of the output on three streams, two "
+                        "slots, copies of one step overlapping another step's compute")},
         "gpu_launches": args.steps * (5 if cfg.keep > 0 and cfg.n_hosts > 1 else 1),
         "clocks": clk,
     }
