@@ -265,44 +265,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (TB > 0) issue_s(1, 0);
         ptx::umma_commit(&bars[K_EMPTY + 0]);
       }
+      // A thread's shared-memory access (an mbarrier check included) right
+      // after it issued UMMAs waits until they have read their operands, so
+      // every check between two UMMA runs lets the tensor core drain.  The
+      // checks are therefore grouped at the head of each run.
       for (int j = 0; ok && j < Tmax; ++j) {
         const int s = j % kVStages;
         if (!ptx::mbar_spin_bounded(&bars[V_FULL + s], (j / kVStages) & 1, gabort, kWaitLimitNs)) {
           record_failure(p.status, 54 + s, j);
           break;
         }
+        // K(j+1), read by this iteration's S MMAs, is checked here with V(j)
+        const bool k_next = j + 1 < Tmax;
+        if (k_next && !(ok = wait_k(j + 1))) break;
         ptx::tc_fence_after();
-        bool k_next = false;   // K(j+1) waited for
         for (int i = 0; i < 2 && ok; ++i) {
           if (j >= T[i]) continue;
           const uint32_t tP = tmem + 128 * i;
+          const uint32_t tOi = tmem + 256 + 128 * i;
           const uint64_t v = dV + s * kTile16;
-          // P_i(j) arrives in two 64-column halves; PV on the first half
-          // overlaps the softmax's exponentials of the second
-          for (int half = 0; half < 2 && ok; ++half) {
-            if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i + half], j & 1, gabort,
+          // P_i(j) arrives in two 64-column halves; PV on the first half may
+          // overlap the softmax's exponentials of the second.  When the second
+          // half is already there both go as one run.
+          if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i], j & 1, gabort, kWaitLimitNs)) {
+            record_failure(p.status, 56 + 2 * i, j);
+            ok = false;
+            break;
+          }
+          const uint32_t acc0 = j > 0 ? 1u : 0u;
+          if (ptx::mbar_test_wait(ptx::smem_u32(&bars[P_FULL + 2 * i + 1]), j & 1)) {
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              ptx::umma_bf16_ts(tOi, tP + kk * 8, v + ((kk * 2048) >> 4), idesc_pv,
+                                kk > 0 ? 1u : acc0);
+          } else {
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              ptx::umma_bf16_ts(tOi, tP + kk * 8, v + ((kk * 2048) >> 4), idesc_pv,
+                                kk > 0 ? 1u : acc0);
+            if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i + 1], j & 1, gabort,
                                         kWaitLimitNs)) {
-              record_failure(p.status, 56 + 2 * i + half, j);
+              record_failure(p.status, 57 + 2 * i, j);
               ok = false;
               break;
             }
             ptx::tc_fence_after();
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              const int kk = half * 4 + k4;
-              ptx::umma_bf16_ts(tmem + 256 + 128 * i, tP + kk * 8, v + ((kk * 2048) >> 4),
-                                idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 4; kk < 8; ++kk)
+              ptx::umma_bf16_ts(tOi, tP + kk * 8, v + ((kk * 2048) >> 4), idesc_pv, 1u);
           }
-          if (!ok) break;
           // V(j)'s last reader is PV_B(j) (or PV_A(j) when tile B has no tile j):
           // release its slot now, before the next S MMA, so its reload starts early
           if (i == 1 || j >= T[1]) ptx::umma_commit(&bars[V_EMPTY + s]);
           if (j + 1 < T[i]) {
-            if (!k_next) {
-              if (!(ok = wait_k(j + 1))) break;
-              k_next = true;
-            }
             issue_s(i, j + 1);
           } else {
             ptx::umma_commit(&bars[O_FINAL + i]);
