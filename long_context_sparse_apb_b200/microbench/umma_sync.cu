@@ -18,30 +18,30 @@ enum Mode {
   kSplitWaits,       // 4 UMMAs, test_wait, 4 UMMAs, test_wait, commit
   kIdleThenWait,     // + 1500 cycles idle on the clock, then test_wait
   kIdleOnly,         // + 1500 cycles idle on the clock
+  kBranch,           // + a data-dependent branch (no memory access)
   kTwoIssuers,       // two issuing warps, each as kTestWait (16 UMMAs per iteration in all)
   kNumModes
 };
 
-__device__ __forceinline__ void umma_run(int n, uint32_t d, uint64_t dA, uint64_t dB,
-                                         uint32_t idesc) {
-  // straight-line runs of 4 or 8 (a branch between UMMAs slows the stream)
-  if (n == 8) {
+__device__ __forceinline__ void umma8(uint32_t d, uint64_t dA, uint64_t dB, uint32_t idesc) {
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t off = ((kk & 3) * 32) >> 4;
-      ptx::umma_bf16_ss(d, dA + off, dB + off, idesc, 1u);
-    }
-  } else {
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = ((kk & 3) * 32) >> 4;
+    ptx::umma_bf16_ss(d, dA + off, dB + off, idesc, 1u);
+  }
+}
+__device__ __forceinline__ void umma4(uint32_t d, uint64_t dA, uint64_t dB, uint32_t idesc) {
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t off = ((kk & 3) * 32) >> 4;
-      ptx::umma_bf16_ss(d, dA + off, dB + off, idesc, 1u);
-    }
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint32_t off = ((kk & 3) * 32) >> 4;
+    ptx::umma_bf16_ss(d, dA + off, dB + off, idesc, 1u);
   }
 }
 
-__global__ void __launch_bounds__(128, 1) umma_sync(int mode, int iters, long long* out,
-                                                     unsigned* err) {
+// One instantiation per mode, so that the issue loop holds no branch on the
+// mode (a branch inside the stream has a cost of its own, see kBranch).
+template <int MODE>
+__global__ void __launch_bounds__(128, 1) umma_sync(int iters, long long* out, unsigned* err) {
   extern __shared__ uint8_t raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)raw + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t bar[5];   // 0, 1: commits of issuer 0 / 1; 2: a completed barrier; 3, 4: drains
@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(128, 1) umma_sync(int mode, int iters, long lo
   if (threadIdx.x == 0) ptx::mbar_arrive(&bar[2]);   // phase 0 of bar[2] completes
   __syncthreads();
   const uint32_t tmem = tm;
-  const bool two = mode == kTwoIssuers;
+  constexpr bool two = MODE == kTwoIssuers;
   if ((warp == 1 || (two && warp == 2)) && lane == 0) {
     const int me = warp - 1;
     const uint32_t idesc = ptx::idesc_bf16_f32(128, 128, 0);
@@ -77,43 +77,46 @@ __global__ void __launch_bounds__(128, 1) umma_sync(int mode, int iters, long lo
     const uint32_t d = tmem + 256 * me;
     uint64_t* cb = &bar[me];
     bool ok = true;
+    uint32_t acc = 0;
     const long long t0 = clock64();
     for (int it = 0; it < iters; ++it) {
-      if (mode == kSplitWaits) {
-        umma_run(4, d, dA, dB, idesc);
+      if (MODE == kSplitWaits) {
+        umma4(d, dA, dB, idesc);
         ok &= ptx::mbar_spin_bounded(&bar[2], 0, &zero, 1000000000ull);
-        umma_run(4, d, dA, dB, idesc);
+        umma4(d, dA, dB, idesc);
         ok &= ptx::mbar_spin_bounded(&bar[2], 0, &zero, 1000000000ull);
         ptx::umma_commit(cb);
         continue;
       }
-      umma_run(8, d, dA, dB, idesc);
+      umma8(d, dA, dB, idesc);
       ptx::umma_commit(cb);
-      if (mode == kTestWait || mode == kTwoIssuers) {
+      if (MODE == kTestWait || MODE == kTwoIssuers) {
         ok &= ptx::mbar_spin_bounded(&bar[2], 0, &zero, 1000000000ull);
-      } else if (mode == kTryWait) {
+      } else if (MODE == kTryWait) {
         ok &= ptx::mbar_wait_bounded(&bar[2], 0, &zero, 1000000000ull);
-      } else if (mode == kLoadVolatile) {
+      } else if (MODE == kLoadVolatile) {
         ok &= flag == 0u;
-      } else if (mode == kLoadAcquire) {
+      } else if (MODE == kLoadAcquire) {
         uint32_t v;
         asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];"
                      : "=r"(v)
                      : "r"(ptx::smem_u32((const void*)&flag))
                      : "memory");
         ok &= v == 0u;
-      } else if (mode == kIdleThenWait || mode == kIdleOnly) {
+      } else if (MODE == kIdleThenWait || MODE == kIdleOnly) {
         const long long t = clock64();
         while (clock64() - t < 1500) {
         }
-        if (mode == kIdleThenWait) ok &= ptx::mbar_spin_bounded(&bar[2], 0, &zero, 1000000000ull);
+        if (MODE == kIdleThenWait) ok &= ptx::mbar_spin_bounded(&bar[2], 0, &zero, 1000000000ull);
+      } else if (MODE == kBranch) {
+        if ((clock64() & 7) == 3) acc += 1;   // data-dependent, no memory access
       }
     }
     const long long t1 = clock64();
     // every MMA of this thread completes before TMEM is freed
     ptx::umma_commit(&bar[3 + me]);
     ok &= ptx::mbar_spin_bounded(&bar[3 + me], 0, &zero, 2000000000ull);
-    if (blockIdx.x == 0) out[me] = t1 - t0;
+    if (blockIdx.x == 0) out[me] = t1 - t0 + (acc == 0xffffffffu);
     if (!ok) atomicOr(err, 1u);
   }
   ptx::tc_fence_before();
@@ -124,6 +127,24 @@ __global__ void __launch_bounds__(128, 1) umma_sync(int mode, int iters, long lo
   }
 }
 
+template <int MODE>
+int run_mode(const char* name, int sms, long long* d, unsigned* err) {
+  const int smem = 48 * 1024 + 1024;
+  cudaFuncSetAttribute(umma_sync<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int iters = 2000;
+  cudaMemset(d, 0, 2 * sizeof(long long));
+  umma_sync<MODE><<<sms, 128, smem>>>(iters, d, err);
+  const cudaError_t e = cudaDeviceSynchronize();
+  long long h[2];
+  cudaMemcpy(h, d, sizeof(h), cudaMemcpyDeviceToHost);
+  unsigned herr;
+  cudaMemcpy(&herr, err, 4, cudaMemcpyDeviceToHost);
+  printf("%-40s: %7.1f cycles per iteration (8 UMMAs of one issuer = 512)", name, (double)h[0] / iters);
+  if (MODE == kTwoIssuers) printf(", second issuer %.1f (16 UMMAs in all = 1024)", (double)h[1] / iters);
+  printf("%s%s\n", herr ? " WAIT FAILED" : "", e != cudaSuccess ? cudaGetErrorString(e) : "");
+  return (herr != 0u) || (e != cudaSuccess);
+}
+
 int main() {
   int sms;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, 0);
@@ -132,27 +153,16 @@ int main() {
   cudaMalloc(&d, 2 * sizeof(long long));
   cudaMalloc(&err, 4);
   cudaMemset(err, 0, 4);
-  const int smem = 48 * 1024 + 1024;
-  cudaFuncSetAttribute(umma_sync, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  const char* names[kNumModes] = {
-      "8 UMMA + commit", "+ test_wait (completed barrier)", "+ try_wait (completed barrier)",
-      "+ ld.volatile.shared", "+ ld.acquire.shared", "4 UMMA, test_wait, 4 UMMA, test_wait",
-      "+ 1500 cycles idle, then test_wait", "+ 1500 cycles idle", "two issuers, each + test_wait"};
   int rc = 0;
-  for (int mode = 0; mode < kNumModes; ++mode) {
-    const int iters = 2000;
-    cudaMemset(d, 0, 2 * sizeof(long long));
-    umma_sync<<<sms, 128, smem>>>(mode, iters, d, err);
-    const cudaError_t e = cudaDeviceSynchronize();
-    long long h[2];
-    cudaMemcpy(h, d, sizeof(h), cudaMemcpyDeviceToHost);
-    unsigned herr;
-    cudaMemcpy(&herr, err, 4, cudaMemcpyDeviceToHost);
-    const double per = (double)h[0] / iters;
-    printf("%-40s: %7.1f cycles per iteration (8 UMMAs of one issuer = 512)", names[mode], per);
-    if (mode == kTwoIssuers) printf(", second issuer %.1f (16 UMMAs in all = 1024)", (double)h[1] / iters);
-    printf("%s%s\n", herr ? " WAIT FAILED" : "", e != cudaSuccess ? cudaGetErrorString(e) : "");
-    rc |= (herr != 0u) || (e != cudaSuccess);
-  }
+  rc |= run_mode<kPlain>("8 UMMA + commit", sms, d, err);
+  rc |= run_mode<kTestWait>("+ test_wait (completed barrier)", sms, d, err);
+  rc |= run_mode<kTryWait>("+ try_wait (completed barrier)", sms, d, err);
+  rc |= run_mode<kLoadVolatile>("+ ld.volatile.shared", sms, d, err);
+  rc |= run_mode<kLoadAcquire>("+ ld.acquire.shared", sms, d, err);
+  rc |= run_mode<kSplitWaits>("4 UMMA, test_wait, 4 UMMA, test_wait", sms, d, err);
+  rc |= run_mode<kIdleThenWait>("+ 1500 cycles idle, then test_wait", sms, d, err);
+  rc |= run_mode<kIdleOnly>("+ 1500 cycles idle", sms, d, err);
+  rc |= run_mode<kBranch>("+ data-dependent branch", sms, d, err);
+  rc |= run_mode<kTwoIssuers>("two issuers, each + test_wait", sms, d, err);
   return rc;
 }
