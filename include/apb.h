@@ -139,6 +139,19 @@ apb_status apb_build_passing(const apb_config* cfg, const void* k, const void* v
                              const int32_t* idx, void* pass_k, void* pass_v,
                              void* stream);
 
+/* Steps 1 and 2 with the passing block emitted straight from the selection
+ * (the fusion of selection and gather): the same scores, idx and selection
+ * rule as apb_score_compress, and pass_k / pass_v exactly as
+ * apb_build_passing writes them, in two launches (score; top-k + gather).
+ *   pass_k, pass_v [H*keep, Hkv, d] bf16 (out), 16-byte aligned; both NULL
+ *   only when keep == 0.
+ * Other arguments and the workspace as for apb_score_compress. */
+apb_status apb_score_compress_pass(const apb_config* cfg, const void* q, const void* k,
+                                   const void* v, const float* w1, const float* b1,
+                                   const float* w2, const float* b2, float* scores, int32_t* idx,
+                                   void* pass_k, void* pass_v, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
 /* Step 3 (main features: computation over anchor, passing and local block;
  * the passing block is not kept afterwards).  For host h, local row i
  * (t = h*n + i) and q head j (g = j / G):

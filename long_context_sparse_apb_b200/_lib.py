@@ -41,6 +41,8 @@ _lib.apb_score_compress.argtypes = [ctypes.POINTER(Config)] + [_P] * 10 + [ctype
 _lib.apb_score_compress.restype = ctypes.c_int
 _lib.apb_score_compress_query_aware.argtypes = _lib.apb_score_compress.argtypes
 _lib.apb_score_compress_query_aware.restype = ctypes.c_int
+_lib.apb_score_compress_pass.argtypes = [ctypes.POINTER(Config)] + [_P] * 12 + [ctypes.c_size_t, _P]
+_lib.apb_score_compress_pass.restype = ctypes.c_int
 _lib.apb_prefill_workspace_bytes.argtypes = [ctypes.POINTER(Config)]
 _lib.apb_prefill_workspace_bytes.restype = ctypes.c_size_t
 _lib.apb_prefill.argtypes = [ctypes.POINTER(Config)] + [_P] * 10 + [ctypes.c_size_t, _P]
@@ -171,6 +173,38 @@ def score_compress(c: Config, q, k, v, w1, b1, w2, b2, scores=None, idx=None, wo
             _stream(stream))
     _check(st, "apb_score_compress_query_aware" if query_aware else "apb_score_compress")
     return idx, scores
+
+
+def score_compress_pass(c: Config, q, k, v, w1, b1, w2, b2, pass_k, pass_v, scores=None,
+                        idx=None, workspace=None, stream=None) -> torch.Tensor:
+    """apb_score_compress_pass: score, top-k and the passing-block gather (the
+    gather in the top-k launch); fills pass_k / pass_v [H*keep, Hkv, d] and
+    returns idx [H, Hkv, keep] int32."""
+    N, hq, hkv, d = _dims(c)
+    _want(q, "q", torch.bfloat16, (N, hq, d))
+    _want(k, "k", torch.bfloat16, (N, hkv, d))
+    _want(v, "v", torch.bfloat16, (N, hkv, d))
+    _want(w1, "w1", torch.float32, (hkv, c.mlp_hidden, 3 * d))
+    _want(b1, "b1", torch.float32, (hkv, c.mlp_hidden))
+    _want(w2, "w2", torch.float32, (hkv, c.mlp_hidden))
+    _want(b2, "b2", torch.float32, (hkv,))
+    _want(pass_k, "pass_k", torch.bfloat16, (c.n_hosts * c.keep, hkv, d))
+    _want(pass_v, "pass_v", torch.bfloat16, (c.n_hosts * c.keep, hkv, d))
+    if scores is not None:
+        _want(scores, "scores", torch.float32, (hkv, N))
+    if idx is None:
+        idx = torch.empty((c.n_hosts, hkv, c.keep), dtype=torch.int32, device=q.device)
+    _want(idx, "idx", torch.int32, (c.n_hosts, hkv, c.keep))
+    if workspace is None:
+        workspace = new_workspace(c, q.device)
+    has = idx.numel() > 0
+    st = _lib.apb_score_compress_pass(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(w1),
+                                      _ptr(b1), _ptr(w2), _ptr(b2), _ptr(scores),
+                                      _ptr(idx) if has else None, _ptr(pass_k) if has else None,
+                                      _ptr(pass_v) if has else None, _ptr(workspace),
+                                      workspace.numel(), _stream(stream))
+    _check(st, "apb_score_compress_pass")
+    return idx
 
 
 def score_compress_static(c: Config, q, k, v, w1, b1, w2, b2, idx=None, stream=None):
@@ -387,8 +421,8 @@ def selftest_wait_timeout(workspace, limit_us: int, stream=None):
 
 
 class Prefill:
-    """One APB prefill over preallocated device buffers: score + compress,
-    build the passing block, block attention.  Buffers are allocated once (by
+    """One APB prefill over preallocated device buffers: score + compress
+    with the passing block built in the top-k launch, then block attention.  Buffers are allocated once (by
     torch) and reused by every call."""
 
     def __init__(self, c: Config, device="cuda"):
@@ -402,9 +436,8 @@ class Prefill:
         self.out = torch.empty((N, hq, d), dtype=torch.bfloat16, device=device)
 
     def __call__(self, q, k, v, w1, b1, w2, b2, stream=None):
-        score_compress(self.c, q, k, v, w1, b1, w2, b2, idx=self.idx, workspace=self.workspace,
-                       stream=stream)
-        build_passing(self.c, k, v, self.idx, self.pass_k, self.pass_v, stream=stream)
+        score_compress_pass(self.c, q, k, v, w1, b1, w2, b2, self.pass_k, self.pass_v,
+                            idx=self.idx, workspace=self.workspace, stream=stream)
         block_attention(self.c, q, k, v, self.pass_k, self.pass_v, out=self.out,
                         workspace=self.workspace, stream=stream)
         return self.out
@@ -487,9 +520,8 @@ class StreamedPrefill:
 
     Per step (streams ordered by events): the H2D stream copies the weights,
     then host 0, 1, ... (q, k, v rows); one compute stream compresses host h
-    (apb_score_compress and apb_build_passing on host h's rows with a
-    one-host config, writing rows [h*keep, (h+1)*keep) of the passing
-    buffers) once its rows are in; two attention streams take hosts in turn
+    (apb_score_compress_pass on host h's rows with a one-host config,
+    writing rows [h*keep, (h+1)*keep) of the passing buffers) once its rows are in; two attention streams take hosts in turn
     (apb_block_attention_range for host h once its rows and the compressed
     blocks of hosts 0..h-1 are in place), so one host's launch fills the
     tail of the other's; the D2H stream copies host h's output rows out.
@@ -565,12 +597,11 @@ class StreamedPrefill:
                 for h in range(H - 1):
                     rows = slice(h * n, (h + 1) * n)
                     self.comp.wait_event(sl["ev_in"][h])
-                    score_compress(self.c1, x["q"][rows], x["k"][rows], x["v"][rows], x["w1"],
-                                   x["b1"], x["w2"], x["b2"], idx=sl["idx"][h],
-                                   workspace=sl["ws_comp"], stream=self.comp)
-                    build_passing(self.c1, x["k"][rows], x["v"][rows], sl["idx"][h],
-                                  sl["pass_k"][h * keep:(h + 1) * keep],
-                                  sl["pass_v"][h * keep:(h + 1) * keep], stream=self.comp)
+                    score_compress_pass(self.c1, x["q"][rows], x["k"][rows], x["v"][rows],
+                                        x["w1"], x["b1"], x["w2"], x["b2"],
+                                        sl["pass_k"][h * keep:(h + 1) * keep],
+                                        sl["pass_v"][h * keep:(h + 1) * keep], idx=sl["idx"][h],
+                                        workspace=sl["ws_comp"], stream=self.comp)
                     sl["ev_pass"][h].record(self.comp)
             sl["ev_done"][0].record(self.comp)
         for h in range(H):

@@ -80,16 +80,21 @@ size_t apb_workspace_bytes(const apb_config* cfg) {
 
 namespace {
 
+// pass_k / pass_v non-NULL: the passing block is built in the top-k launch.
 apb_status score_compress_impl(const char* who, bool query_aware, const apb_config* cfg,
                                const void* q, const void* k, const void* v, const float* w1,
                                const float* b1, const float* w2, const float* b2, float* scores,
-                               int32_t* idx, void* workspace, size_t ws_bytes, void* stream) {
+                               int32_t* idx, void* pass_k, void* pass_v, void* workspace,
+                               size_t ws_bytes, void* stream) {
   apb::Shape s;
   apb_status st = check_config(cfg, &s);
   if (st != APB_OK) return st;
   if (!q || !k || !v || !w1 || !b1 || !w2 || !b2 || !workspace)
     return fail(APB_ERR_INVALID_ARG, "%s: NULL input or workspace", who);
   if (s.keep > 0 && !idx) return fail(APB_ERR_INVALID_ARG, "%s: idx is NULL", who);
+  const bool fused = pass_k || pass_v;
+  if (fused && s.keep > 0 && (!pass_k || !pass_v || !aligned16(pass_k) || !aligned16(pass_v)))
+    return fail(APB_ERR_INVALID_ARG, "%s: pass_k / pass_v NULL or not 16-byte aligned", who);
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w1) || !aligned16(workspace) ||
       (scores && !aligned16(scores)) || (idx && !aligned16(idx)))
     return fail(APB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
@@ -112,7 +117,8 @@ apb_status score_compress_impl(const char* who, bool query_aware, const apb_conf
   if (why) return fail(APB_ERR_CUDA, "score: %s", why);
   if (e != cudaSuccess) return cuda_fail(e, "score kernel");
   if (s.keep > 0) {
-    e = apb::launch_topk(s, sc, idx, cs);
+    e = fused ? apb::launch_topk_gather(s, sc, idx, k, v, pass_k, pass_v, cs)
+              : apb::launch_topk(s, sc, idx, cs);
     if (e != cudaSuccess) return cuda_fail(e, "top-k kernel");
   }
   return APB_OK;
@@ -129,7 +135,16 @@ apb_status apb_score_compress(const apb_config* cfg, const void* q, const void* 
                               int32_t* idx, void* workspace, size_t ws_bytes,
                               void* stream) {
   return score_compress_impl("apb_score_compress", false, cfg, q, k, v, w1, b1, w2, b2, scores,
-                             idx, workspace, ws_bytes, stream);
+                             idx, nullptr, nullptr, workspace, ws_bytes, stream);
+}
+
+apb_status apb_score_compress_pass(const apb_config* cfg, const void* q, const void* k,
+                                   const void* v, const float* w1, const float* b1,
+                                   const float* w2, const float* b2, float* scores, int32_t* idx,
+                                   void* pass_k, void* pass_v, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  return score_compress_impl("apb_score_compress_pass", false, cfg, q, k, v, w1, b1, w2, b2,
+                             scores, idx, pass_k, pass_v, workspace, ws_bytes, stream);
 }
 
 apb_status apb_score_compress_query_aware(const apb_config* cfg, const void* q, const void* k,
@@ -138,7 +153,7 @@ apb_status apb_score_compress_query_aware(const apb_config* cfg, const void* q, 
                                           int32_t* idx, void* workspace, size_t ws_bytes,
                                           void* stream) {
   return score_compress_impl("apb_score_compress_query_aware", true, cfg, q, k, v, w1, b1, w2, b2,
-                             scores, idx, workspace, ws_bytes, stream);
+                             scores, idx, nullptr, nullptr, workspace, ws_bytes, stream);
 }
 
 apb_status apb_build_passing(const apb_config* cfg, const void* k, const void* v,
@@ -313,10 +328,9 @@ apb_status apb_prefill(const apb_config* cfg, const void* q, const void* k, cons
                           &why);
     if (why) return fail(APB_ERR_CUDA, "score: %s", why);
     if (e != cudaSuccess) return cuda_fail(e, "score kernel");
-    e = apb::launch_topk(s1, scores, idx, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "top-k kernel");
-    e = apb::launch_gather(s1, k, v, idx, ws + L.pass_k, ws + L.pass_v, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "gather kernel");
+    // selection and the passing-block gather in one launch
+    e = apb::launch_topk_gather(s1, scores, idx, k, v, ws + L.pass_k, ws + L.pass_v, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k + gather kernel");
   }
   apb::HostRange r{0, s.H, 1, 0, 0, 0, s.N, s.N};
   const char* why = nullptr;

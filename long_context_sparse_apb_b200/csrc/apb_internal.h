@@ -48,6 +48,10 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
                          const float* b2, float* scores, void* wsplit, float* qbias,
                          DeviceStatus* status, cudaStream_t st, const char** why);
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* idx, cudaStream_t st);
+// Top-k and the passing-block gather in one launch (pass_k / pass_v as in
+// launch_gather).
+cudaError_t launch_topk_gather(const Shape& s, const float* scores, int32_t* idx, const void* k,
+                               const void* v, void* pass_k, void* pass_v, cudaStream_t st);
 cudaError_t launch_gather(const Shape& s, const void* k, const void* v, const int32_t* idx,
                           void* pass_k, void* pass_v, cudaStream_t st);
 // Hosts [hb, he) of one attention launch and where their rows sit: row of

@@ -10,6 +10,11 @@
 // output is ascending and ties go to the lower position -- deterministic.
 // The block's keys are staged in shared memory when they fit, else re-read
 // from global memory (L2-resident) in every pass.
+//
+// The fused form (launch_topk_gather) then builds the (host, kv head)'s
+// compressed block straight from the selection: the same CTA copies the
+// selected K and V rows into the passing buffers (one launch and no second
+// read of the indices from another kernel).
 #include "apb_internal.h"
 
 namespace apb {
@@ -50,9 +55,19 @@ __device__ __forceinline__ int block_exclusive_count(bool flag, int* warp_sums, 
   return res;
 }
 
+struct GatherArgs {
+  const uint4* k;   // [N, Hkv, d] bf16 as 16-byte chunks
+  const uint4* v;
+  uint4* pass_k;    // [H * keep, Hkv, d]
+  uint4* pass_v;
+  int chunks_per_row;
+};
+
+template <bool GATHER>
 __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict__ scores,
                                                         int32_t* __restrict__ idx, int n, int keep,
-                                                        long long N, int Hkv, bool stage) {
+                                                        long long N, int Hkv, bool stage,
+                                                        GatherArgs ga) {
   extern __shared__ uint32_t skeys[];
   __shared__ int hist[256];
   __shared__ int warp_sums[kThreads / 32 + 1];
@@ -126,21 +141,57 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
     written += sel_tot;
     eq_seen += eq_tot;
   }
+  if (GATHER) {
+    // pass[h*keep + r, g, :] = src[idx[h, g, r], g, :] for K and V; the
+    // indices were written above by this CTA (visible after the barrier;
+    // read with plain loads, not the read-only path).  Consecutive threads
+    // copy consecutive 16-byte chunks of a row.
+    __syncthreads();
+    const int cpr = ga.chunks_per_row;
+    const long long row0 = (long long)h * keep;
+    for (int e = threadIdx.x; e < keep * cpr; e += kThreads) {
+      const int r = e / cpr, c = e - r * cpr;
+      const long long t = out[r];
+      uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+      if (t >= 0 && t < N) {
+        const long long src = (t * Hkv + g) * cpr + c;
+        a = __ldg(ga.k + src);
+        b = __ldg(ga.v + src);
+      }
+      const long long dst = ((row0 + r) * Hkv + g) * cpr + c;
+      ga.pass_k[dst] = a;
+      ga.pass_v[dst] = b;
+    }
+  }
+}
+
+template <bool GATHER>
+cudaError_t launch(const Shape& s, const float* scores, int32_t* idx, GatherArgs ga,
+                   cudaStream_t st) {
+  const bool stage = s.n <= kMaxSmemKeys;
+  const size_t smem = stage ? (size_t)s.n * sizeof(uint32_t) : 0;
+  if (stage) {
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel<GATHER>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(s.Hkv, s.H);
+  topk_kernel<GATHER><<<grid, kThreads, smem, st>>>(scores, idx, s.n, s.keep, s.N, s.Hkv, stage,
+                                                    ga);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const Shape& s, const float* scores, int32_t* idx, cudaStream_t st) {
-  const bool stage = s.n <= kMaxSmemKeys;
-  const size_t smem = stage ? (size_t)s.n * sizeof(uint32_t) : 0;
-  if (stage) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  dim3 grid(s.Hkv, s.H);
-  topk_kernel<<<grid, kThreads, smem, st>>>(scores, idx, s.n, s.keep, s.N, s.Hkv, stage);
-  return cudaGetLastError();
+  return launch<false>(s, scores, idx, GatherArgs{}, st);
+}
+
+cudaError_t launch_topk_gather(const Shape& s, const float* scores, int32_t* idx, const void* k,
+                               const void* v, void* pass_k, void* pass_v, cudaStream_t st) {
+  GatherArgs ga{static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+                static_cast<uint4*>(pass_k), static_cast<uint4*>(pass_v), s.d * 2 / 16};
+  return launch<true>(s, scores, idx, ga, st);
 }
 
 }  // namespace apb

@@ -140,3 +140,24 @@ def test_host_range_and_query_aware_checks():
     st = apb._lib.apb_score_compress_query_aware(ctypes.byref(bad), *([FAKE] * 8), FAKE, FAKE,
                                                  1 << 30, None)
     assert st == apb.APB_ERR_UNSUPPORTED
+
+
+def test_score_compress_pass_checks():
+    # the fused call takes the score call's checks plus its own on the
+    # passing buffers, all before any launch
+    c = apb.make_config(inputs.TINY)
+    ws = apb.workspace_bytes(c)
+    args = [FAKE] * 8   # q, k, v, w1, b1, w2, b2, scores
+    st = apb._lib.apb_score_compress_pass(ctypes.byref(c), *args, FAKE, None, FAKE, FAKE, ws, None)
+    assert st == apb.APB_ERR_INVALID_ARG                       # pass_k NULL
+    st = apb._lib.apb_score_compress_pass(ctypes.byref(c), *args, FAKE, FAKE, MISALIGNED, FAKE,
+                                          ws, None)
+    assert st == apb.APB_ERR_INVALID_ARG                       # pass_v misaligned
+    st = apb._lib.apb_score_compress_pass(ctypes.byref(c), *args, None, FAKE, FAKE, FAKE, ws, None)
+    assert st == apb.APB_ERR_INVALID_ARG                       # idx NULL with keep > 0
+    bad = apb.make_config(inputs.TINY, head_dim=96)
+    st = apb._lib.apb_score_compress_pass(ctypes.byref(bad), *args, FAKE, FAKE, FAKE, FAKE, ws,
+                                          None)
+    assert st == apb.APB_ERR_UNSUPPORTED
+    st = apb._lib.apb_score_compress_pass(ctypes.byref(c), *args, FAKE, FAKE, FAKE, FAKE, 64, None)
+    assert st == apb.APB_ERR_INVALID_ARG                       # workspace too small

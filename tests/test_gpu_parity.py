@@ -269,6 +269,34 @@ def test_single_call_prefill_equals_three_calls(apb, cfg):
     assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
 
 
+@pytest.mark.parametrize("cfg", [inputs.TINY,
+                                 inputs.TINY.replace(n_hosts=5, block_len=300, anchor_len=75,
+                                                     keep=130, n_q_heads=10, n_kv_heads=2,
+                                                     head_dim=128, seed=13),
+                                 inputs.TINY.replace(keep=512, seed=14)],
+                         ids=["tiny", "ragged_g5", "keep_n"])
+def test_score_compress_pass_equals_separate_calls(apb, cfg):
+    # selection and gather in one launch: idx, scores and both passing
+    # buffers equal the two-call path bit for bit
+    x = inputs.generate(cfg)
+    xd = _to_dev(x)
+    c = apb.make_config(cfg)
+    N, hq, hkv, d = c.n_hosts * c.block_len, c.n_q_heads, c.n_kv_heads, c.head_dim
+    w = (xd["w1"], xd["b1"], xd["w2"], xd["b2"])
+    ref_scores = torch.empty((hkv, N), dtype=torch.float32, device="cuda")
+    ref_idx, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, scores=ref_scores)
+    ref_pk, ref_pv = apb.build_passing(c, xd["k"], xd["v"], ref_idx)
+    scores = torch.empty_like(ref_scores)
+    pk = torch.full_like(ref_pk, float("nan"))
+    pv = torch.full_like(ref_pv, float("nan"))
+    idx = apb.score_compress_pass(c, xd["q"], xd["k"], xd["v"], *w, pk, pv, scores=scores)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(scores.view(torch.int32), ref_scores.view(torch.int32))
+    assert torch.equal(pk.view(torch.int16), ref_pk.view(torch.int16))
+    assert torch.equal(pv.view(torch.int16), ref_pv.view(torch.int16))
+
+
 def test_topk_unstaged_path_large_block(apb):
     # blocks above 48K tokens re-read their scores from global memory in every
     # radix pass instead of staging them in shared memory
