@@ -57,21 +57,28 @@ __device__ constexpr bool kPolyPairs[8] = {
     APB_POLY_OF_8 > 0, APB_POLY_OF_8 > 4, APB_POLY_OF_8 > 2, APB_POLY_OF_8 > 6,
     APB_POLY_OF_8 > 1, APB_POLY_OF_8 > 5, APB_POLY_OF_8 > 3, APB_POLY_OF_8 > 7};
 
+#ifndef APB_K_STAGES
+#define APB_K_STAGES 2
+#endif
+#ifndef APB_V_STAGES
+#define APB_V_STAGES 3
+#endif
+constexpr int kKStages = APB_K_STAGES;
+constexpr int kVStages = APB_V_STAGES;   // V is released later than K: one more stage of prefetch
+static_assert(kKStages + kVStages == 5, "shared memory holds Q_A, Q_B and five K/V stages");
+
 enum Bar {
   Q_FULL = 0,
-  K_FULL = 1,    // kKStages
-  K_EMPTY = 3,   // kKStages
-  V_FULL = 5,    // kVStages
-  V_EMPTY = 8,   // kVStages
-  S_FULL = 11,   // per query tile (A, B)
-  P_FULL = 13,   // per query tile and 64-column half: 13 + 2 * tile + half
-  O_FINAL = 17,  // per query tile
-  DRAIN = 19,
-  NUM_BARS = 20
+  K_FULL = 1,                       // kKStages
+  K_EMPTY = K_FULL + kKStages,      // kKStages
+  V_FULL = K_EMPTY + kKStages,      // kVStages
+  V_EMPTY = V_FULL + kVStages,      // kVStages
+  S_FULL = V_EMPTY + kVStages,      // per query tile (A, B)
+  P_FULL = S_FULL + 2,              // per query tile and 64-column half: + 2 * tile + half
+  O_FINAL = P_FULL + 4,             // per query tile
+  DRAIN = O_FINAL + 2,
+  NUM_BARS = DRAIN + 1
 };
-
-constexpr int kKStages = 2;
-constexpr int kVStages = 3;   // V is released later than K: one more stage of prefetch
 
 template <int D>
 struct Layout {
@@ -187,7 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !skip) {
-      int lastK[kKStages] = {-1, -1}, lastV[kVStages] = {-1, -1, -1};   // last load parity per slot
+      int lastK[kKStages], lastV[kVStages];   // last load parity per slot (-1: never loaded)
+      for (int i = 0; i < kKStages; ++i) lastK[i] = -1;
+      for (int i = 0; i < kVStages; ++i) lastV[i] = -1;
       ptx::mbar_arrive_expect_tx(&bars[Q_FULL], (TB > 0 ? 2 : 1) * L::kTile);
       for (int i = 0; i < (TB > 0 ? 2 : 1); ++i) {
 #pragma unroll
