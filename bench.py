@@ -430,7 +430,8 @@ def run_gpu(args, cfg):
                         "PrefillPipeline (blocks shorter than 4096 rows): pinned H2D copies, one "
                         "apb_prefill call and the D2H copy of the output on three streams, two "
                         "slots, copies of one step overlapping another step's compute")},
-        "gpu_launches": args.steps * (5 if cfg.keep > 0 and cfg.n_hosts > 1 else 1),
+        # per apb_prefill: weight split, score, top-k with the gather, attention
+        "gpu_launches": args.steps * (4 if cfg.keep > 0 and cfg.n_hosts > 1 else 1),
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
@@ -558,7 +559,9 @@ def run_sharded(args, cfg):
                 "exchange_bytes_per_rank": 2 * sp.count * cfg.keep * cfg.n_kv_heads
                 * cfg.head_dim * 2,
                 "e2e": None, "e2e_note": "host-buffer end-to-end is measured in the default mode",
-                "gpu_launches": args.steps * (cfg.n_hosts // world) * (4 if cfg.keep else 2)
+                # per owned host: weight split, score, top-k (with the gather
+                # when keep > 0); one attention launch per step
+                "gpu_launches": args.steps * (cfg.n_hosts // world) * (3 if cfg.keep else 2)
                 + args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -612,7 +615,7 @@ def run_heads(args, cfg):
                 "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": cdict, "e2e": None,
                 "e2e_note": "host-buffer end-to-end is measured in the default mode",
-                "gpu_launches": args.steps * (5 if cfg.keep else 3), "clocks": clk}
+                "gpu_launches": args.steps * (4 if cfg.keep else 3), "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -8,10 +8,11 @@ One process per GPU.  Rank r of W owns H/W hosts, either round-robin (hosts
 r, r+W, r+2W, ...: the default, which balances the work, since a host's
 attention grows with its index through the passing block) or contiguous
 (hosts [r*H/W, (r+1)*H/W)).  Per step, on each rank:
-  1. for every owned host: score + top-k (apb_score_compress on that host's
-     block) and its compressed block, written straight into the host's rows
-     [h*keep, (h+1)*keep) of a full token-major passing buffer
-     (apb_build_passing);
+  1. for every owned host: score + top-k and its compressed block, written
+     straight into the host's rows [h*keep, (h+1)*keep) of a full token-major
+     passing buffer (apb_score_compress_pass: the gather runs in the top-k
+     launch; the query-aware variant takes apb_score_compress_query_aware +
+     apb_build_passing);
   2. all-gathers of the passing buffer's K and V rows that leave every
      host's block in host order: round-robin, one per round i over the rows
      of hosts [i*W, (i+1)*W) (rank r contributes host i*W + r); contiguous,
@@ -144,6 +145,12 @@ class ShardedPrefill:
             qs = q[i * n:(i + 1) * n]
             ks = kv_k[A + i * n:A + (i + 1) * n]
             vs = kv_v[A + i * n:A + (i + 1) * n]
+            if keep > 0 and not query_aware:
+                apb.score_compress_pass(self.c1, qs, ks, vs, w1, b1, w2, b2,
+                                        self.pass_k[h * keep:(h + 1) * keep],
+                                        self.pass_v[h * keep:(h + 1) * keep], idx=self.idx[i],
+                                        workspace=self.workspace, stream=stream)
+                continue
             apb.score_compress(self.c1, qs, ks, vs, w1, b1, w2, b2, idx=self.idx[i],
                                workspace=self.workspace, stream=stream, query_aware=query_aware)
             if keep > 0:
