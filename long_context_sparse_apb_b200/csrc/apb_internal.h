@@ -10,6 +10,10 @@
 namespace apb {
 
 // Status block at the start of every workspace.
+// "where" codes: 40-75 the attention kernel (named kWhere* in
+// attention.cu), 80-90 the score kernel (80/82 + CTA rank: weight / k,v
+// producer; 84 accumulator free; 85 chunk operands; 86 + rank q converter
+// slots; 88 + rank epilogue; 90 shared-memory alignment check).
 struct DeviceStatus {
   uint32_t sticky;     // OR of error bits since last clear
   uint32_t abort;      // set inside a launch once one CTA gave up

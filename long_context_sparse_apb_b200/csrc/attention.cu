@@ -66,6 +66,17 @@ __device__ constexpr bool kPolyPairs[8] = {
 constexpr int kKStages = APB_K_STAGES;
 constexpr int kVStages = APB_V_STAGES;   // V is released later than K: one more stage of prefetch
 static_assert(kKStages + kVStages == 5, "shared memory holds Q_A, Q_B and five K/V stages");
+static_assert(kKStages <= 3 && kVStages <= 3, "failure codes leave room for three slots each");
+
+// Failure codes ("where" in the status block) of this kernel's waits.
+constexpr uint32_t kWhereKEmpty = 40;   // producer, + K slot
+constexpr uint32_t kWhereVEmpty = 45;   // producer, + V slot
+constexpr uint32_t kWhereQ = 50;        // issuer: Q_A, Q_B landed
+constexpr uint32_t kWhereKFull = 51;    // issuer, + K slot
+constexpr uint32_t kWhereVFull = 54;    // issuer, + V slot
+constexpr uint32_t kWhereS = 60;        // softmax, + query tile
+constexpr uint32_t kWhereO = 63;        // epilogue, + query tile
+constexpr uint32_t kWhereP = 70;        // issuer, + 2 * query tile + half
 
 enum Bar {
   Q_FULL = 0,
@@ -208,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ks = j % kKStages, vs = j % kVStages;
         const uint32_t kpar = (j / kKStages) & 1, vpar = (j / kVStages) & 1;
         if (!ptx::mbar_wait_bounded(&bars[K_EMPTY + ks], kpar ^ 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 40 + ks, j);
+          record_failure(p.status, kWhereKEmpty + ks, j);
           break;
         }
         ptx::mbar_arrive_expect_tx(&bars[K_FULL + ks], L::kTile);
@@ -216,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         local_row0, p.anchor_row0);
         lastK[ks] = (int)kpar;
         if (!ptx::mbar_wait_bounded(&bars[V_EMPTY + vs], vpar ^ 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 42 + vs, j);
+          record_failure(p.status, kWhereVEmpty + vs, j);
           break;
         }
         ptx::mbar_arrive_expect_tx(&bars[V_FULL + vs], L::kTile);
@@ -259,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait_k = [&](int jj) -> bool {
         if (!ptx::mbar_spin_bounded(&bars[K_FULL + jj % kKStages], (jj / kKStages) & 1, gabort,
                                     kWaitLimitNs)) {
-          record_failure(p.status, 51 + jj % kKStages, jj);
+          record_failure(p.status, kWhereKFull + jj % kKStages, jj);
           return false;
         }
         ptx::tc_fence_after();
@@ -267,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       bool ok = ptx::mbar_wait_bounded(&bars[Q_FULL], 0, gabort, kWaitLimitNs);
-      if (!ok) record_failure(p.status, 50, 0);
+      if (!ok) record_failure(p.status, kWhereQ, 0);
       if (ok) ok = wait_k(0);
       if (ok) {
         issue_s(0, 0);
@@ -281,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < Tmax; ++j) {
         const int s = j % kVStages;
         if (!ptx::mbar_spin_bounded(&bars[V_FULL + s], (j / kVStages) & 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, 54 + s, j);
+          record_failure(p.status, kWhereVFull + s, j);
           break;
         }
         // K(j+1), read by this iteration's S MMAs, is checked here with V(j)
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // overlap the softmax's exponentials of the second.  When the second
           // half is already there both go as one run.
           if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i], j & 1, gabort, kWaitLimitNs)) {
-            record_failure(p.status, 56 + 2 * i, j);
+            record_failure(p.status, kWhereP + 2 * i, j);
             ok = false;
             break;
           }
@@ -316,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 kk > 0 ? 1u : acc0);
             if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i + 1], j & 1, gabort,
                                         kWaitLimitNs)) {
-              record_failure(p.status, 57 + 2 * i, j);
+              record_failure(p.status, kWhereP + 2 * i + 1, j);
               ok = false;
               break;
             }
@@ -355,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < T; ++j) {
       ok = ptx::mbar_wait_bounded(&bars[S_FULL + i], j & 1, gabort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) record_failure(p.status, 60 + i, j);
+        if (lane == 0) record_failure(p.status, kWhereS + i, j);
         ok = false;
         break;
       }
@@ -450,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && T > 0) {
       ok = ptx::mbar_wait_bounded(&bars[O_FINAL + i], 0, gabort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) record_failure(p.status, 63 + i, T);
+        if (lane == 0) record_failure(p.status, kWhereO + i, T);
         ok = false;
       }
       if (ok) {
