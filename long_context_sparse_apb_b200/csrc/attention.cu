@@ -77,6 +77,7 @@ constexpr uint32_t kWhereVFull = 54;    // issuer, + V slot
 constexpr uint32_t kWhereS = 60;        // softmax, + query tile
 constexpr uint32_t kWhereO = 63;        // epilogue, + query tile
 constexpr uint32_t kWhereP = 70;        // issuer, + 2 * query tile + half
+constexpr uint32_t kWherePV0 = 74;      // softmax, + query tile (rare rescale path)
 
 enum Bar {
   Q_FULL = 0,
@@ -88,7 +89,8 @@ enum Bar {
   P_FULL = S_FULL + 2,              // per query tile and 64-column half: + 2 * tile + half
   O_FINAL = P_FULL + 4,             // per query tile
   DRAIN = O_FINAL + 2,
-  NUM_BARS = DRAIN + 1
+  PV0_DONE = DRAIN + 1,             // per query tile: PV_i(j) on the first P half has run
+  NUM_BARS = PV0_DONE + 2
 };
 
 template <int D>
@@ -319,12 +321,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < 8; ++kk)
               ptx::umma_bf16_ts(tOi, tP + kk * 8, v + ((kk * 2048) >> 4), idesc_pv,
                                 kk > 0 ? 1u : acc0);
+            ptx::umma_commit(&bars[PV0_DONE + i]);
           } else {
             ptx::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               ptx::umma_bf16_ts(tOi, tP + kk * 8, v + ((kk * 2048) >> 4), idesc_pv,
                                 kk > 0 ? 1u : acc0);
+            ptx::umma_commit(&bars[PV0_DONE + i]);
             if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i + 1], j & 1, gabort,
                                         kWaitLimitNs)) {
               record_failure(p.status, kWhereP + 2 * i + 1, j);
@@ -371,8 +375,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       ptx::tc_fence_after();
-      uint32_t sr[128];
-      APB_TMEM_LD128(tS, sr);
       // visible columns of this row in this tile
       int lim;
       if (j < na) {
@@ -382,53 +384,63 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         lim = (j == T - 1) ? row + 1 : kRows;
       }
-      if (lim < kRows) {
+      // Lazy maximum.  m is the tile-0 row maximum and moves only when a
+      // 64-column half would otherwise produce probabilities beyond 2^64
+      // (detected from the half's row sum, which the pass computes anyway):
+      // P = 2^(s*scale - m) stays finite in bf16 and the fp32 sums of O and l
+      // keep ~2^60 of headroom, and the tiles after the first need no pass
+      // over the scores for their maximum.  The result is that of the
+      // running-maximum softmax up to rounding (O and l share the base m).
+      uint32_t sr[64];
+      APB_TMEM_LD32(tS, sr);
+      APB_TMEM_LD32(tS + 32, sr + 32);
+      if (lim < 64) {
 #pragma unroll
-        for (int c = 0; c < kRows; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c >= lim) sr[c] = 0xff800000u;   // -inf
       }
-      float mx[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x)
-        mx[x] = fmaxf(__uint_as_float(sr[2 * x]), __uint_as_float(sr[2 * x + 1]));
-#pragma unroll
-      for (int c = 16; c < kRows; c += 2)
-        mx[(c >> 1) & 7] = ptx::fmax3(mx[(c >> 1) & 7], __uint_as_float(sr[c]),
-                                      __uint_as_float(sr[c + 1]));
-      const float tmax = fmaxf(ptx::fmax3(mx[0], mx[1], mx[2]),
-                               fmaxf(ptx::fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float m_tile = tmax * p.scale_log2;
-      float alpha = 1.f;
-      bool rescale = false;
       if (j == 0) {
-        m = m_tile;
-      } else if (m_tile > m + kRescaleThreshold) {
-        alpha = ptx::ex2(m - m_tile);
-        m = m_tile;
-        l *= alpha;
-        rescale = true;
-      }
-      const float mneg = -m;
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        // the first tile's maximum, the second half read 32 columns at a time
+        float mx[8];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if (half == 1) {
-          // reload the second half of S (cheaper than keeping 64 more
-          // registers alive through the first half)
-          APB_TMEM_LD32(tS + 64, sr + 64);
-          APB_TMEM_LD32(tS + 96, sr + 96);
-          if (lim < kRows) {
+        for (int x = 0; x < 8; ++x)
+          mx[x] = fmaxf(__uint_as_float(sr[2 * x]), __uint_as_float(sr[2 * x + 1]));
 #pragma unroll
-            for (int c = 64; c < kRows; ++c)
-              if (c >= lim) sr[c] = 0xff800000u;   // -inf
+        for (int c = 16; c < 64; c += 2)
+          mx[(c >> 1) & 7] = ptx::fmax3(mx[(c >> 1) & 7], __uint_as_float(sr[c]),
+                                        __uint_as_float(sr[c + 1]));
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          uint32_t t[32];
+          APB_TMEM_LD32(tS + 64 + 32 * part, t);
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            const int c = 64 + 32 * part + x;
+            const float a0 = c < lim ? __uint_as_float(t[x]) : -INFINITY;
+            const float a1 = c + 1 < lim ? __uint_as_float(t[x + 1]) : -INFINITY;
+            mx[(x >> 1) & 7] = ptx::fmax3(mx[(x >> 1) & 7], a0, a1);
           }
         }
-        uint32_t pk[32];
+        m = fmaxf(ptx::fmax3(mx[0], mx[1], mx[2]),
+                  fmaxf(ptx::fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+            p.scale_log2;
+      }
+      auto half_max = [&]() -> float {   // this half's maximum (log2 units)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 64; c += 2)
+          mx[(c >> 1) & 3] = ptx::fmax3(mx[(c >> 1) & 3], __uint_as_float(sr[c]),
+                                        __uint_as_float(sr[c + 1]));
+        return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+      };
+      // exponentials and row sum of the 64 scores in sr (columns 64*half..)
+      auto exps = [&](float mneg, uint32_t (&pk)[32], float (&acc)[4]) {
+#pragma unroll
+        for (int x = 0; x < 4; ++x) acc[x] = 0.f;
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) {
-          const int c = half * 32 + cc;
           float x0, x1, p0, p1;
-          ptx::ffma2_scalar(x0, x1, __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]),
+          ptx::ffma2_scalar(x0, x1, __uint_as_float(sr[2 * cc]), __uint_as_float(sr[2 * cc + 1]),
                             p.scale_log2, mneg);
           if (kPolyPairs[cc & 7]) {
             ptx::exp2_poly2(p0, p1, x0, x1);      // part of the pairs on the FMA pipe
@@ -436,26 +448,89 @@ __global__ void __launch_bounds__(kThreads, 1)
             p0 = ptx::ex2(x0);
             p1 = ptx::ex2(x1);
           }
-          ptx::fadd2_acc(sum[(c & 1) * 2], sum[(c & 1) * 2 + 1], p0, p1);
+          ptx::fadd2_acc(acc[(cc & 1) * 2], acc[(cc & 1) * 2 + 1], p0, p1);
           pk[cc] = ptx::pack_bf16x2(p0, p1);
         }
-        // O_i is stable here (the commit that signalled S_i(j) covers
-        // PV_i(j-1)); it must be rescaled before PV_i(j) starts on half 0
-        if (half == 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            APB_TMEM_LD32(tO + 32 * c, o);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            APB_TMEM_ST32(tO + 32 * c, o);
-          }
-        }
-        APB_TMEM_ST32(tS + 32 * half, pk);
-        ptx::tmem_st_wait();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars[P_FULL + 2 * i + half]);
+      };
+      constexpr float kSumLimit = 18446744073709551616.0f;   // 2^64
+      float sum[4];
+      uint32_t pk[32];
+      // ---- first half
+      exps(-m, pk, sum);
+      bool rescale = false;
+      float alpha = 1.f;
+      if (!((sum[0] + sum[1]) + (sum[2] + sum[3]) < kSumLimit)) {   // rare (and NaN-safe)
+        const float m_new = fmaxf(m, half_max());
+        alpha = ptx::ex2(m - m_new);
+        m = m_new;
+        l *= alpha;
+        rescale = true;
+        exps(-m, pk, sum);
       }
+      // O_i is stable here (the commit that signalled S_i(j) covers
+      // PV_i(j-1)); it must be rescaled before PV_i(j) starts on half 0
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          APB_TMEM_LD32(tO + 32 * c, o);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+          APB_TMEM_ST32(tO + 32 * c, o);
+        }
+      }
+      APB_TMEM_ST32(tS, pk);
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars[P_FULL + 2 * i]);
+      // ---- second half
+      APB_TMEM_LD32(tS + 64, sr);
+      APB_TMEM_LD32(tS + 96, sr + 32);
+      if (lim < kRows) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (64 + c >= lim) sr[c] = 0xff800000u;   // -inf
+      }
+      float sum1[4];
+      exps(-m, pk, sum1);
+      const bool big = !((sum1[0] + sum1[1]) + (sum1[2] + sum1[3]) < kSumLimit);
+      if (__any_sync(0xffffffffu, big)) {
+        // rare: m moves after the first half's probabilities went out, so O
+        // (which PV_i(j) on the first half is adding to) is rescaled once that
+        // PV has run, before the second half's
+        const bool w = ptx::mbar_wait_bounded(&bars[PV0_DONE + i], j & 1, gabort, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, w)) {
+          if (lane == 0) record_failure(p.status, kWherePV0 + i, j);
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        float a1 = 1.f;
+        if (big) {
+          const float m_new = fmaxf(m, half_max());
+          a1 = ptx::ex2(m - m_new);
+          m = m_new;
+          l *= a1;
+#pragma unroll
+          for (int x = 0; x < 4; ++x) sum[x] *= a1;
+          exps(-m, pk, sum1);
+        }
+        __syncwarp();   // the rows that moved m rejoin before the warp-collective TMEM access
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          APB_TMEM_LD32(tO + 32 * c, o);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * a1);
+          APB_TMEM_ST32(tO + 32 * c, o);
+        }
+      }
+      APB_TMEM_ST32(tS + 32, pk);
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars[P_FULL + 2 * i + 1]);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) sum[x] += sum1[x];
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     }
     if (ok && T > 0) {

@@ -297,6 +297,33 @@ def test_score_compress_pass_equals_separate_calls(apb, cfg):
     assert torch.equal(pv.view(torch.int16), ref_pv.view(torch.int16))
 
 
+@pytest.mark.parametrize("mult", [14.0, 60.0], ids=["x_about_80", "x_about_345"])
+def test_scores_far_above_the_first_tiles(apb, mult):
+    # the softmax keeps the first tile's row maximum as its base and moves it
+    # only when a 64-column half's probabilities would pass 2^64: plant one
+    # key whose logits lie ~80 or ~345 (log2 units) above everything the rows
+    # saw before, for kv head 0 in the first half of host 1's first local
+    # tile and for kv head 1 in its second half, so both of those paths run
+    # (the second after the first half's probabilities have gone to the
+    # tensor core); at ~345 the probabilities would overflow without them
+    cfg = inputs.TINY.replace(seed=41)
+    x = inputs.generate(cfg)
+    n, G, d = cfg.block_len, cfg.group, cfg.head_dim
+    h = 1
+    gen = torch.Generator().manual_seed(41)
+    q = x["q"].float()
+    k = x["k"].float()
+    # host h's queries: one direction per q head (|u|^2 ~ d) plus a little noise
+    u = torch.randn(cfg.n_q_heads, d, generator=gen)
+    q[h * n:(h + 1) * n] = u[None] + 0.1 * torch.randn(n, cfg.n_q_heads, d, generator=gen)
+    for g, local in ((0, 10), (1, 72)):          # local tile 0, column 10 / column 72
+        ug = u[g * G:(g + 1) * G].mean(0)
+        k[h * n + local, g] = mult * ug          # logit ~ mult * (d / 2) / sqrt(d) * log2(e)
+    x["q"] = q.to(torch.bfloat16)
+    x["k"] = k.to(torch.bfloat16)
+    _full_parity(apb, cfg, x)
+
+
 def test_topk_unstaged_path_large_block(apb):
     # blocks above 48K tokens re-read their scores from global memory in every
     # radix pass instead of staging them in shared memory
