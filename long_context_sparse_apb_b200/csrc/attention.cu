@@ -392,8 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // over the scores for their maximum.  The result is that of the
       // running-maximum softmax up to rounding (O and l share the base m).
       uint32_t sr[64];
-      APB_TMEM_LD32(tS, sr);
-      APB_TMEM_LD32(tS + 32, sr + 32);
+      APB_TMEM_LD64(tS, sr);
       if (lim < 64) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
@@ -484,8 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars[P_FULL + 2 * i]);
       // ---- second half
-      APB_TMEM_LD32(tS + 64, sr);
-      APB_TMEM_LD32(tS + 96, sr + 32);
+      APB_TMEM_LD64(tS + 64, sr);
       if (lim < kRows) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
