@@ -623,11 +623,17 @@ def run_heads(args, cfg):
 
 
 def apb_kernel_rev() -> str:
-    """Hash of the attention kernel source: ncu traffic counters only apply to
-    the revision they were taken on."""
+    """Hash of the attention kernel source with comments and blank lines
+    removed: ncu traffic counters only apply to the code they were taken on
+    (a comment edit does not change it)."""
     import hashlib
+    import re
     p = os.path.join(ROOT, "long_context_sparse_apb_b200", "csrc", "attention.cu")
-    return hashlib.sha1(open(p, "rb").read()).hexdigest()[:12]
+    src = open(p, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+    return hashlib.sha1(code.encode()).hexdigest()[:12]
 
 
 def main():

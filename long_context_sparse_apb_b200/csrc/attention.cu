@@ -387,9 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Lazy maximum.  m is the tile-0 row maximum and moves only when a
       // 64-column half would otherwise produce probabilities beyond 2^64
       // (detected from the half's row sum, which the pass computes anyway):
-      // P = 2^(s*scale - m) stays finite in bf16 and the fp32 sums of O and l
-      // keep ~2^60 of headroom, and the tiles after the first need no pass
-      // over the scores for their maximum.  The result is that of the
+      // P = 2^(s*scale - m) <= 2^64 stays finite in bf16, and summed over up to
+      // 2^20 keys it keeps O and l inside the fp32 range for |V| up to ~2^40;
+      // the tiles after the first need no pass over the scores for their
+      // maximum.  The result is that of the
       // running-maximum softmax up to rounding (O and l share the base m).
       uint32_t sr[64];
       APB_TMEM_LD64(tS, sr);
