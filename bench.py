@@ -622,18 +622,22 @@ def run_heads(args, cfg):
         dist.destroy_process_group()
 
 
-def apb_kernel_rev() -> str:
-    """Hash of the attention kernel source with comments and blank lines
-    removed: ncu traffic counters only apply to the code they were taken on
-    (a comment edit does not change it)."""
+def source_rev(src: str) -> str:
+    """Hash of C++ source with comments, blank lines and trailing blanks
+    removed."""
     import hashlib
     import re
-    p = os.path.join(ROOT, "long_context_sparse_apb_b200", "csrc", "attention.cu")
-    src = open(p, encoding="utf-8").read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     src = re.sub(r"//[^\n]*", "", src)
     code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
     return hashlib.sha1(code.encode()).hexdigest()[:12]
+
+
+def apb_kernel_rev() -> str:
+    """Revision of the attention kernel's code: ncu traffic counters only
+    apply to the code they were taken on (a comment edit does not change it)."""
+    p = os.path.join(ROOT, "long_context_sparse_apb_b200", "csrc", "attention.cu")
+    return source_rev(open(p, encoding="utf-8").read())
 
 
 def main():
