@@ -95,6 +95,8 @@ SMALL = [
     (5, 513, 200, 32, 0, 8, 2, 128),     # keep 0, ragged n and anchor
     (3, 257, 33, 33, 257, 10, 2, 64),    # keep = n, G = 5
     (4, 384, 96, 16, 130, 4, 1, 128),    # passing tail of 2 rows per 128-tile
+    (2, 200, 50, 10, 40, 6, 2, 128),     # G = 3 (one partial head group)
+    (3, 150, 40, 8, 20, 7, 1, 64),       # G = 7 (a full and a partial head group)
 ]
 
 
