@@ -500,13 +500,13 @@ def run_sharded(args, cfg):
     all-gathered over NCCL, each rank attends its hosts.  Strong scaling:
     value = tokens of the one sequence / max-over-ranks step time."""
     from long_context_sparse_apb_b200 import _lib as apb
-    from long_context_sparse_apb_b200.sharded import ShardedPrefill, nccl_all_gather
+    from long_context_sparse_apb_b200.sharded import ShardedPrefill, tensor_all_gather
 
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     c = apb.make_config(cfg)
     sp = ShardedPrefill(c, rank, world, device=dev,
-                        all_gather=nccl_all_gather() if world > 1 else None)
+                        all_gather=tensor_all_gather() if world > 1 else None)
     loc = {k: v.to(dev) for k, v in inputs.generate_local(
         cfg, sp.first, sp.first + sp.count * sp.stride, sp.stride).items()}
     w = (loc["w1"], loc["b1"], loc["w2"], loc["b2"])

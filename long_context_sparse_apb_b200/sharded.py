@@ -85,25 +85,15 @@ def head_slice(x: dict, n_q_heads: int, n_kv_heads: int, gb: int, ge: int) -> di
     return out
 
 
-def nccl_all_gather(group=None) -> Callable[[torch.Tensor, torch.Tensor], None]:
-    """In-place all-gather of a rank's chunk into the full buffer (NCCL):
-    `chunk` must be this rank's slice of `full`."""
+def tensor_all_gather(group=None) -> Callable[[torch.Tensor, torch.Tensor], None]:
+    """In-place all-gather of a rank's chunk into the full buffer through
+    torch.distributed.all_gather_into_tensor: NCCL between GPUs, gloo between
+    CPU ranks.  `chunk` must be this rank's slot of `full` (slot `rank` of
+    `world` equal parts)."""
     import torch.distributed as dist
 
     def gather(full: torch.Tensor, chunk: torch.Tensor) -> None:
         dist.all_gather_into_tensor(full, chunk, group=group)
-    return gather
-
-
-def list_all_gather(group=None) -> Callable[[torch.Tensor, torch.Tensor], None]:
-    """The same exchange through torch.distributed.all_gather (any backend,
-    used by the CPU tests with gloo)."""
-    import torch.distributed as dist
-
-    def gather(full: torch.Tensor, chunk: torch.Tensor) -> None:
-        world = dist.get_world_size(group)
-        parts = list(full.chunk(world, dim=0))
-        dist.all_gather(parts, chunk.clone(), group=group)
     return gather
 
 

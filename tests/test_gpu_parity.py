@@ -109,6 +109,17 @@ def test_small_shapes_every_row(apb, shape):
     _full_parity(apb, cfg)
 
 
+@pytest.mark.parametrize("d,G", [(128, 4), (64, 2)])
+def test_star_configuration_long_anchor(apb, d, G):
+    # The Star-style mask the bench times next to APB (anchor = the whole
+    # first block, no passing block), with H >= 3 and an anchor of 18 KV tiles
+    # ending in a ragged one (2300 = 17 * 128 + 124): every row of every host
+    cfg = inputs.APBConfig("star", n_hosts=3, block_len=2300, anchor_len=2300, query_len=64,
+                           keep=0, n_q_heads=2 * G, n_kv_heads=2, head_dim=d, seed=41 + d,
+                           rope_theta=5e5, needles_per_host=4)
+    _full_parity(apb, cfg)
+
+
 def test_deterministic_repeat(apb):
     cfg = inputs.TINY.replace(n_hosts=3, block_len=640, anchor_len=160, keep=100)
     xd = _to_dev(inputs.generate(cfg))

@@ -1,12 +1,34 @@
 """Host-sharded prefill (several GPUs in the pages' design) emulated on one
 GPU: W ranks run their steps on their own rank-local buffers, the all-gather
 of the compressed blocks is emulated by copying each rank's chunk into every
-rank's passing buffer, and the concatenated outputs must equal the
-single-GPU path bit for bit (same kernels, same arithmetic per tile)."""
+rank's passing buffer.  Each rank's output is checked against the fp64
+oracle (selection within the tie rule, attention within the stated
+tolerance on the ranks' own index set) and against the single-GPU path bit
+for bit (same kernels, same arithmetic per tile).  Likewise for the
+kv-head split."""
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from long_context_sparse_apb_b200 import inputs
+
+from _parity import check_topk, compare_attention, f32np, oracle_scores
+
+
+def _oracle_check(cfg, x, idx_all, out_of_host, heads=None):
+    """idx_all [H, Hkv, keep] global positions chosen by the GPU ranks;
+    out_of_host(h) -> the ranks' output rows of host h [n, nh, d] (heads
+    `heads`, default all)."""
+    if cfg.keep > 0:
+        check_topk(idx_all, oracle_scores(cfg, x), cfg)
+    k, v = f32np(x["k"]), f32np(x["v"])
+    pk, pv = oracle.passing_blocks(k, v, idx_all.astype(np.int64))
+    n = cfg.block_len
+    for h in range(cfg.n_hosts):
+        o_ref, _, _ = oracle.host_attention(f32np(x["q"][h * n:(h + 1) * n]), np.arange(n), h, k,
+                                            v, pk, pv, n, cfg.anchor_len, cfg.keep, heads=heads)
+        compare_attention(f32np(out_of_host(h)), o_ref, f"{cfg.name} host {h}")
 
 pytestmark = pytest.mark.gpu
 
@@ -44,12 +66,17 @@ def test_sharded_equals_single_gpu(cfg, world, order):
                     dst.pass_k[rows].copy_(src.pass_k[rows])
                     dst.pass_v[rows].copy_(src.pass_v[rows])
     n = cfg.block_len
+    rows_of_host = {}
+    idx_all = np.zeros((cfg.n_hosts, cfg.n_kv_heads, keep), dtype=np.int64)
     for sp, loc in zip(ranks, locs):
         out = sp.attend(loc["q"], loc["k"], loc["v"])
         torch.cuda.synchronize()
         assert apb.device_status(sp.workspace) == apb.APB_OK
         for i, h in enumerate(sp.hosts):
             assert torch.equal(out[i * n:(i + 1) * n], ref[h * n:(h + 1) * n]), (order, h)
+            rows_of_host[h] = out[i * n:(i + 1) * n].clone()
+            idx_all[h] = sp.idx[i, 0].cpu().numpy() + h * n      # one-host calls: local rows
+    _oracle_check(cfg, x, idx_all, lambda h: rows_of_host[h])
 
 
 @pytest.mark.parametrize("world", [2])
@@ -67,6 +94,8 @@ def test_kv_head_sharding_equals_single_gpu(world):
     full = apb.Prefill(apb.make_config(cfg))
     ref = full(xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"], xd["b2"]).clone()
     G = cfg.group
+    n, H = cfg.block_len, cfg.n_hosts
+    outs, idx_all = [], np.zeros((H, cfg.n_kv_heads, cfg.keep), dtype=np.int64)
     for r in range(world):
         gb, ge = kv_head_range(cfg.n_kv_heads, r, world)
         loc = head_slice(xd, cfg.n_q_heads, cfg.n_kv_heads, gb, ge)
@@ -76,3 +105,11 @@ def test_kv_head_sharding_equals_single_gpu(world):
         torch.cuda.synchronize()
         assert torch.equal(out, ref[:, gb * G:ge * G])
         assert torch.equal(run.idx, full.idx[:, gb:ge])
+        outs.append(out.clone())
+        # the one-call path compresses hosts 0..H-2 only (the last host's
+        # block has no reader); the oracle check needs every host's indices
+        idx_all[:H - 1, gb:ge] = run.idx[:H - 1].cpu().numpy()
+    sh = torch.cat(outs, dim=1)               # heads back in order
+    s_ref = oracle_scores(cfg, x)
+    idx_all[H - 1] = oracle.compress_indices(s_ref, H, n, cfg.keep)[H - 1]
+    _oracle_check(cfg, x, idx_all, lambda h: sh[h * n:(h + 1) * n])

@@ -12,7 +12,9 @@ host prefix for the passing block, a wrong tie rule) fails at least one:
   ``torch.nn.functional.scaled_dot_product_attention`` in float64
   (H = 1; keep = n with no anchor; a full-block anchor with keep = 0; host 0
   of any configuration), an additive-bias identity for duplicated keys,
-  softmax normalisation and invariance to the passing block's row order.
+  softmax normalisation and invariance to the passing block's row order;
+* visible-pair count: an explicit per-slot visibility mask on tiny cases, and
+  the number of keys the oracle's attention spreads its weight over.
 """
 import json
 import math
@@ -290,6 +292,49 @@ def test_visible_pairs_count():
     c = inputs.LLAMA8B_128K
     assert visible_pairs(c.n_hosts, c.block_len, c.anchor_len, c.keep) == 2_248_212_480
     assert visible_pairs(1, 10, 3, 2) == 55
+
+
+def _visible_mask_count(H, n, A, keep):
+    """Brute force: one boolean per (host, local query, key slot), the key
+    slots being the A anchor rows, the H*keep rows of the gathered compressed
+    blocks and the n rows of the host's own block; each rule of "APB 的主要功能"
+    (anchor for hosts >= 1, the blocks of earlier hosts only, local causal
+    with the diagonal) is applied slot by slot."""
+    total = 0
+    for h in range(H):
+        for i in range(n):
+            mask = np.zeros(A + H * keep + n, dtype=bool)
+            for a in range(A):
+                mask[a] = h >= 1
+            for r in range(H * keep):
+                mask[A + r] = (r // keep) < h          # block of host r // keep, before h
+            for c in range(n):
+                mask[A + H * keep + c] = c <= i
+            total += int(mask.sum())
+    return total
+
+
+@pytest.mark.parametrize("H,n,A,keep", [(3, 7, 3, 2), (4, 5, 5, 0), (3, 6, 0, 6), (2, 9, 2, 1)])
+def test_visible_pairs_brute_force(H, n, A, keep):
+    assert visible_pairs(H, n, A, keep) == _visible_mask_count(H, n, A, keep)
+
+
+def test_visible_pairs_equals_attended_keys():
+    """With q = 0 every visible key gets the same logit, so the oracle's
+    attention has exp(lse) = number of keys the row attends; summed over the
+    rows of every host this is the visible-pair count of one q head."""
+    H, n, A, keep, d = 3, 7, 3, 2, 4
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal((H * n, 1, d))
+    v = rng.standard_normal((H * n, 1, d))
+    idx = np.stack([np.stack([np.sort(rng.choice(n, keep, replace=False)) + h * n])
+                    for h in range(H)])
+    pk, pv = passing_blocks(k, v, idx)
+    total = 0.0
+    for h in range(H):
+        _, lse, _ = host_attention(np.zeros((n, 1, d)), np.arange(n), h, k, v, pk, pv, n, A, keep)
+        total += np.exp(lse).sum()
+    assert round(total) == visible_pairs(H, n, A, keep) == _visible_mask_count(H, n, A, keep)
 
 
 # ----------------------------------------------------------------- configs

@@ -1,6 +1,8 @@
 """The all-gather of the host-sharded prefill on CPU ranks (gloo, world
-size 2): every rank ends with all ranks' compressed-block rows in host order,
-for both host assignments, and the host sets partition the hosts."""
+size 2): ShardedPrefill.exchange, with the same all_gather_into_tensor call
+the GPU ranks make over NCCL, leaves every rank with all ranks'
+compressed-block rows in host order, for both host assignments; the host
+sets partition the hosts."""
 import os
 import socket
 
@@ -54,19 +56,28 @@ def _free_port():
 def _worker(rank, world, port, q, order):
     os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
                       MASTER_PORT=str(port))
+    import datetime
+
     import torch
     import torch.distributed as dist
-    from long_context_sparse_apb_b200.sharded import exchange_chunks, host_set, list_all_gather
+    from long_context_sparse_apb_b200 import _lib as apb
+    from long_context_sparse_apb_b200.sharded import ShardedPrefill, tensor_all_gather
 
-    dist.init_process_group("gloo")
-    H, keep, hkv, d = 4, 3, 2, 4
-    full = torch.zeros(H * keep, hkv, d)
-    first, count, stride = host_set(H, rank, world, order)
-    for h in range(first, first + count * stride, stride):     # this rank's blocks
-        full[h * keep:(h + 1) * keep] = 100 * h + torch.arange(keep * hkv * d).reshape(keep, hkv, d)
-    for rows, chunk in exchange_chunks(H, keep, rank, world, order):
-        list_all_gather()(full[rows], full[chunk])
-    q.put((rank, full.numpy()))
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    H, n, keep, hkv, d = 4, 16, 3, 2, 64
+    c = apb.make_config(None, n_hosts=H, block_len=n, anchor_len=4, query_len=2, keep=keep,
+                        n_q_heads=4, n_kv_heads=hkv, head_dim=d)
+    # the exchange of the GPU path (all_gather_into_tensor on slices of the
+    # passing buffers), run on CPU tensors between gloo ranks
+    sp = ShardedPrefill(c, rank, world, device="cpu", all_gather=tensor_all_gather(), order=order)
+    sp.pass_k.zero_()
+    sp.pass_v.zero_()
+    for h in sp.hosts:                                         # this rank's blocks
+        blk = 100 * h + torch.arange(keep * hkv * d).reshape(keep, hkv, d)
+        sp.pass_k[h * keep:(h + 1) * keep] = blk.to(torch.bfloat16)
+        sp.pass_v[h * keep:(h + 1) * keep] = (-blk).to(torch.bfloat16)
+    sp.exchange()
+    q.put((rank, sp.pass_k.float().numpy(), sp.pass_v.float().numpy()))
     dist.destroy_process_group()
 
 
@@ -82,9 +93,10 @@ def test_exchange_two_gloo_ranks(order):
     for p in procs:
         p.join(timeout=120)
     assert all(p.exitcode == 0 for p in procs)
-    res = dict(q.get(timeout=5) for _ in range(2))
-    keep, hkv, d = 3, 2, 4
+    res = {r: (k, v) for r, k, v in (q.get(timeout=5) for _ in range(2))}
+    keep, hkv, d = 3, 2, 64
     expect = torch.cat([100 * h + torch.arange(keep * hkv * d).reshape(keep, hkv, d)
-                        for h in range(4)]).float()
+                        for h in range(4)]).to(torch.bfloat16).float()
     for r in range(2):
-        assert torch.equal(torch.from_numpy(res[r]), expect)
+        assert torch.equal(torch.from_numpy(res[r][0]), expect)
+        assert torch.equal(torch.from_numpy(res[r][1]), -expect)
