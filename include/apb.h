@@ -244,11 +244,15 @@ apb_status apb_prefill(const apb_config* cfg, const void* q, const void* k, cons
  *     of scores and 8 MiB of split weights; every GPU that loads the library
  *     keeps them until the process exits.  n_kv_heads * N above the first,
  *     or n_kv_heads * mlp_hidden * 3 * head_dim * 4 bytes above the second,
- *     returns APB_ERR_UNSUPPORTED.  A bounded wait that runs out inside
- *     this variant is not reported (its status block is private).
- *   - The first call on each device looks up the arrays' device addresses
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     returns APB_ERR_UNSUPPORTED with the exceeded limit in
+ *     apb_last_error().  A bounded wait that runs out inside this variant is
+ *     recorded in the library's own status block, which
+ *     apb_score_compress_static_status reads.
+ *   - Every call looks up the arrays' device addresses on the current device
+ *     (cudaGetSymbolAddress, a host-side lookup), so the call works on
+ *     whichever device is current and after cudaDeviceReset; the first call
+ *     on a device should still come before any stream capture (it may load
+ *     the module on that device).
  *   - All calls share the arrays and they keep the last call's contents.
  *     Each call writes every score it reads, so nothing needs clearing, but
  *     two calls whose kernels overlap on the GPU (other streams or threads)
@@ -258,6 +262,20 @@ apb_status apb_score_compress_static(const apb_config* cfg, const void* q, const
                                      const void* v, const float* w1, const float* b1,
                                      const float* w2, const float* b2, int32_t* idx,
                                      void* stream);
+
+/* No counterpart in the paper.  apb_device_status for the fixed status block
+ * of apb_score_compress_static on the current device: synchronises `stream`,
+ * returns APB_ERR_TIMEOUT if one of its kernels recorded a bounded wait that
+ * ran out since the block was last cleared (the top-k that followed then
+ * read incomplete scores: discard idx), else APB_OK.  clear != 0 resets the
+ * block afterwards. */
+apb_status apb_score_compress_static_status(void* stream, int clear);
+
+/* No counterpart in the paper: apb_selftest_wait_timeout run on the fixed
+ * status block of apb_score_compress_static (current device), so that a
+ * caller can check that apb_score_compress_static_status reports a wait that
+ * ran out.  limit_us in [1, 1000000]. */
+apb_status apb_score_compress_static_selftest(uint32_t limit_us, void* stream);
 
 /* No counterpart in the paper: a self-test of the bounded waits every kernel
  * uses.  Launches two CTAs that each wait on an on-chip barrier that nothing

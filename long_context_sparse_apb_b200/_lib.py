@@ -63,6 +63,10 @@ _lib.apb_score_compress_static.argtypes = [ctypes.POINTER(Config)] + [_P] * 9
 _lib.apb_score_compress_static.restype = ctypes.c_int
 _lib.apb_score_compress_static_max_floats.argtypes = []
 _lib.apb_score_compress_static_max_floats.restype = ctypes.c_size_t
+_lib.apb_score_compress_static_status.argtypes = [_P, ctypes.c_int]
+_lib.apb_score_compress_static_status.restype = ctypes.c_int
+_lib.apb_score_compress_static_selftest.argtypes = [ctypes.c_uint32, _P]
+_lib.apb_score_compress_static_selftest.restype = ctypes.c_int
 _lib.apb_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
 _lib.apb_selftest_wait_timeout.restype = ctypes.c_int
 _lib.apb_device_status.argtypes = [_P, _P, ctypes.c_int]
@@ -226,6 +230,19 @@ def score_compress_static(c: Config, q, k, v, w1, b1, w2, b2, idx=None, stream=N
                                         _ptr(idx) if idx.numel() else None, _stream(stream))
     _check(st, "apb_score_compress_static")
     return idx
+
+
+def score_compress_static_status(stream=None, clear=False) -> int:
+    """apb_score_compress_static_status: synchronises the stream and returns
+    APB_ERR_TIMEOUT if a wait inside apb_score_compress_static ran out."""
+    return int(_lib.apb_score_compress_static_status(_stream(stream), 1 if clear else 0))
+
+
+def score_compress_static_selftest(limit_us: int, stream=None):
+    """apb_score_compress_static_selftest: the bounded-wait self-test on the
+    static entry point's own status block."""
+    st = _lib.apb_score_compress_static_selftest(limit_us, _stream(stream))
+    _check(st, "apb_score_compress_static_selftest")
 
 
 def build_passing(c: Config, k, v, idx, pass_k=None, pass_v=None, stream=None):

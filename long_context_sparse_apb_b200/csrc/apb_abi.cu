@@ -9,8 +9,10 @@
 #include "apb_internal.h"
 
 namespace {
-
 thread_local char g_last_error[512] = "";
+}  // namespace
+
+namespace apb {
 
 apb_status fail(apb_status st, const char* fmt, ...) {
   va_list ap;
@@ -19,6 +21,17 @@ apb_status fail(apb_status st, const char* fmt, ...) {
   va_end(ap);
   return st;
 }
+
+apb_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(APB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace apb
+
+namespace {
+
+using apb::cuda_fail;
+using apb::fail;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -60,10 +73,6 @@ apb_status check_config(const apb_config* c, apb::Shape* s) {
 }
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
-
-apb_status cuda_fail(cudaError_t e, const char* what) {
-  return fail(APB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
-}
 
 }  // namespace
 

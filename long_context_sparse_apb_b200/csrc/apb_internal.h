@@ -9,6 +9,12 @@
 
 namespace apb {
 
+// Sets the thread-local message that apb_last_error() returns (printf-style)
+// and returns `st`; cuda_fail does the same for a CUDA runtime error, as
+// APB_ERR_CUDA with "<what>: <CUDA error string>".
+apb_status fail(apb_status st, const char* fmt, ...);
+apb_status cuda_fail(cudaError_t e, const char* what);
+
 // Status block at the start of every workspace.
 // "where" codes: 40-75 the attention kernel (named kWhere* in
 // attention.cu), 80-90 the score kernel (80/82 + CTA rank: weight / k,v
@@ -68,6 +74,12 @@ struct HostRange {
   int h0, count, stride, q_row0, k_row0, anchor_row0;
   long long q_rows, k_rows;
 };
+
+// The bounded-wait self-test on `status` (two CTAs waiting on barriers that
+// nothing completes; CTA 0 gives up after limit_us, CTA 1 through the abort
+// flag); the two waits' durations go to elapsed_ns[0..1].
+cudaError_t launch_wait_selftest(DeviceStatus* status, uint32_t limit_us,
+                                 unsigned long long* elapsed_ns, cudaStream_t st);
 
 // Returns cudaSuccess or an error; sets *why when a TMA descriptor could not
 // be built (reported as APB_ERR_CUDA with a message).

@@ -33,18 +33,33 @@ __global__ void selftest_wait_kernel(DeviceStatus* status, uint64_t short_ns, ui
 }  // namespace
 }  // namespace apb
 
+namespace apb {
+
+cudaError_t launch_wait_selftest(DeviceStatus* status, uint32_t limit_us,
+                                 unsigned long long* elapsed_ns, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(&status->abort, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  const uint64_t short_ns = (uint64_t)limit_us * 1000ull;
+  selftest_wait_kernel<<<2, 32, 0, st>>>(status, short_ns, 20ull * short_ns + 1000000000ull,
+                                         elapsed_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace apb
+
 extern "C" apb_status apb_selftest_wait_timeout(void* workspace, size_t ws_bytes,
                                                 uint32_t limit_us, void* stream) {
   if (!workspace || ws_bytes < apb::kStatusBytes || (reinterpret_cast<uintptr_t>(workspace) & 15))
-    return APB_ERR_INVALID_ARG;
-  if (limit_us == 0 || limit_us > 1000000) return APB_ERR_INVALID_ARG;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    return apb::fail(APB_ERR_INVALID_ARG,
+                     "apb_selftest_wait_timeout: workspace NULL, unaligned or < %zu bytes",
+                     apb::kStatusBytes);
+  if (limit_us == 0 || limit_us > 1000000)
+    return apb::fail(APB_ERR_INVALID_ARG, "apb_selftest_wait_timeout: limit_us=%u not in [1, 1e6]",
+                     limit_us);
   auto* status = static_cast<apb::DeviceStatus*>(workspace);
   // elapsed times of the two waits go to the spare bytes of the status block
   auto* elapsed = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + 64);
-  if (cudaMemsetAsync(&status->abort, 0, sizeof(uint32_t), cs) != cudaSuccess) return APB_ERR_CUDA;
-  const uint64_t short_ns = (uint64_t)limit_us * 1000ull;
-  apb::selftest_wait_kernel<<<2, 32, 0, cs>>>(status, short_ns, 20ull * short_ns + 1000000000ull,
-                                             elapsed);
-  return cudaGetLastError() == cudaSuccess ? APB_OK : APB_ERR_CUDA;
+  const cudaError_t e = apb::launch_wait_selftest(status, limit_us, elapsed,
+                                                  reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? APB_OK : apb::cuda_fail(e, "self-test kernel");
 }
