@@ -22,8 +22,9 @@
 // softmax has read S_A; likewise P_B in S_B.
 // Per KV tile j and query tile i:
 //   S_i(j) = Q_i K(j)^T         tcgen05.mma, A and B from shared memory
-//   softmax_i reads S_i(j), rescales O_i in TMEM when the running max grew by
-//   more than 2^8 (lazy rescaling), writes P_i(j) to TMEM, signals P_FULL_i
+//   softmax_i reads S_i(j), exponentiates against a lazily moved row maximum
+//   (O_i is rescaled in TMEM only when that base moves), writes P_i(j) to
+//   TMEM in two 64-column halves, signals P_FULL_i per half
 //   O_i += P_i(j) V(j)          tcgen05.mma, A = P_i from TMEM, B = V
 // The MMA thread issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while one
 // softmax warpgroup works on its tile the tensor core serves the other.
@@ -47,26 +48,9 @@ constexpr int kRows = 128;                    // query rows per tile = KV rows p
 constexpr int kThreads = 320;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;     // log2 units
-// Which pairs of every 8 take 2^x on the FMA pipe instead of MUFU ex2
-// (balances the two pipes; the rest use ex2.approx).
-#ifndef APB_POLY_OF_8
-#define APB_POLY_OF_8 0
-#endif
-__device__ constexpr bool kPolyPairs[8] = {
-    APB_POLY_OF_8 > 0, APB_POLY_OF_8 > 4, APB_POLY_OF_8 > 2, APB_POLY_OF_8 > 6,
-    APB_POLY_OF_8 > 1, APB_POLY_OF_8 > 5, APB_POLY_OF_8 > 3, APB_POLY_OF_8 > 7};
-
-#ifndef APB_K_STAGES
-#define APB_K_STAGES 2
-#endif
-#ifndef APB_V_STAGES
-#define APB_V_STAGES 3
-#endif
-constexpr int kKStages = APB_K_STAGES;
-constexpr int kVStages = APB_V_STAGES;   // V is released later than K: one more stage of prefetch
+constexpr int kKStages = 2;
+constexpr int kVStages = 3;   // V is released later than K: one more stage of prefetch
 static_assert(kKStages + kVStages == 5, "shared memory holds Q_A, Q_B and five K/V stages");
-static_assert(kKStages <= 3 && kVStages <= 3, "failure codes leave room for three slots each");
 
 // Failure codes ("where" in the status block) of this kernel's waits.
 constexpr uint32_t kWhereKEmpty = 40;   // producer, + K slot
@@ -442,12 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float x0, x1, p0, p1;
           ptx::ffma2_scalar(x0, x1, __uint_as_float(sr[2 * cc]), __uint_as_float(sr[2 * cc + 1]),
                             p.scale_log2, mneg);
-          if (kPolyPairs[cc & 7]) {
-            ptx::exp2_poly2(p0, p1, x0, x1);      // part of the pairs on the FMA pipe
-          } else {
-            p0 = ptx::ex2(x0);
-            p1 = ptx::ex2(x1);
-          }
+          p0 = ptx::ex2(x0);
+          p1 = ptx::ex2(x1);
           ptx::fadd2_acc(acc[(cc & 1) * 2], acc[(cc & 1) * 2 + 1], p0, p1);
           pk[cc] = ptx::pack_bf16x2(p0, p1);
         }

@@ -347,43 +347,5 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair on the FMA pipe (no MUFU): Cody-Waite style reduction
-// x = n + f with n = rint(x) (magic-number rounding), f in [-1/2, 1/2], then
-// 2^f by a degree-3 polynomial fitted here by iteratively reweighted least
-// squares on Chebyshev nodes (max relative error 7.5e-5, below the 2^-9
-// rounding of the bf16 probabilities it feeds), and 2^n added to the
-// exponent field.  x is clamped to >= -125 so the result stays a positive
-// normal number (2^-125 stands for 0 next to row sums >= 1).
-__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
-  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer
-  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
-  constexpr float c2 = 0.2426111251115799f, c3 = 0.05517164617776871f;
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  uint32_t t0b, t1b, p0b, p1b;
-  asm("{\n\t.reg .b64 x, t, n, f, p, m, mn, k;\n\t"
-      "mov.b64 x, {%4, %5};\n\t"
-      "mov.b64 m, {%6, %6};\n\t"
-      "mov.b64 mn, {%7, %7};\n\t"
-      "add.rn.f32x2 t, x, m;\n\t"            // t = x + magic (integer n in low bits)
-      "add.rn.f32x2 n, t, mn;\n\t"           // n = rint(x)
-      "mov.b64 k, {%12, %12};\n\t"
-      "fma.rn.f32x2 f, n, k, x;\n\t"         // f = x - n
-      "mov.b64 p, {%11, %11};\n\t"
-      "mov.b64 k, {%10, %10};\n\t"
-      "fma.rn.f32x2 p, p, f, k;\n\t"         // c3 f + c2
-      "mov.b64 k, {%9, %9};\n\t"
-      "fma.rn.f32x2 p, p, f, k;\n\t"         // (.) f + c1
-      "mov.b64 k, {%8, %8};\n\t"
-      "fma.rn.f32x2 p, p, f, k;\n\t"         // (.) f + c0
-      "mov.b64 {%0, %1}, t;\n\t"
-      "mov.b64 {%2, %3}, p;\n\t}"
-      : "=r"(t0b), "=r"(t1b), "=r"(p0b), "=r"(p1b)
-      : "f"(x0), "f"(x1), "f"(kMagic), "f"(-kMagic), "f"(c0), "f"(c1), "f"(c2), "f"(c3),
-        "f"(-1.0f));
-  y0 = __uint_as_float(p0b + (t0b << 23));
-  y1 = __uint_as_float(p1b + (t1b << 23));
-}
-
 }  // namespace ptx
 }  // namespace apb
