@@ -1,6 +1,8 @@
 """bench.py's multi-rank plumbing on CPU ranks (gloo, world size 2): rank
-setup, barrier, max-over-ranks timing and the per-rank independent sequence
-(weak scaling, no collective on the data path)."""
+setup, barrier, max-over-ranks timing, the default kv-head split of one
+sequence (each rank's inputs are its heads' slice, the slices tile the
+sequence's heads) and the per-rank independent sequence of the replica mode;
+no collective on the data path."""
 import os
 import socket
 
@@ -28,7 +30,10 @@ def _worker(rank, world, port, out):
     bench.barrier(w)
     mx = bench.max_over_ranks(10.0 + rank, w)
     cfg = bench.rank_config(inputs.TINY, r)
-    out.put((rank, mx, cfg.seed))
+    lcfg, lx = bench.local_work(inputs.TINY, "heads", r, w)
+    assert (lcfg.n_kv_heads, lcfg.n_q_heads) == (1, 2)
+    out.put((rank, mx, cfg.seed, lx["q"].float().numpy(), lx["k"].float().numpy(),
+             lx["w1"].numpy()))
     dist.destroy_process_group()
 
 
@@ -39,10 +44,21 @@ def test_two_gloo_ranks():
     procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
-    for p in procs:
-        p.join(timeout=120)
+    try:
+        # read before joining: a child holding unsent queue data cannot exit
+        res = sorted((q.get(timeout=120) for _ in range(2)), key=lambda t: t[0])
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
     assert all(p.exitcode == 0 for p in procs)
-    res = sorted(q.get(timeout=5) for _ in range(2))
-    assert [m for _, m, _ in res] == [11.0, 11.0]          # max over ranks
-    seeds = [s for _, _, s in res]
+    assert [t[1] for t in res] == [11.0, 11.0]             # max over ranks
+    seeds = [t[2] for t in res]
     assert seeds[0] != seeds[1]                             # independent sequences
+    from long_context_sparse_apb_b200 import inputs
+    full = inputs.generate(inputs.TINY)
+    import numpy as np
+    assert np.array_equal(np.concatenate([res[0][3], res[1][3]], axis=1), full["q"].float().numpy())
+    assert np.array_equal(np.concatenate([res[0][4], res[1][4]], axis=1), full["k"].float().numpy())
+    assert np.array_equal(np.concatenate([res[0][5], res[1][5]], axis=0), full["w1"].numpy())

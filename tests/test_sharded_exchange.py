@@ -90,10 +90,15 @@ def test_exchange_two_gloo_ranks(order):
     procs = [ctx.Process(target=_worker, args=(r, 2, port, q, order)) for r in range(2)]
     for p in procs:
         p.start()
-    for p in procs:
-        p.join(timeout=120)
+    try:
+        # read before joining: a child holding unsent queue data cannot exit
+        res = {r: (k, v) for r, k, v in (q.get(timeout=120) for _ in range(2))}
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
     assert all(p.exitcode == 0 for p in procs)
-    res = {r: (k, v) for r, k, v in (q.get(timeout=5) for _ in range(2))}
     keep, hkv, d = 3, 2, 64
     expect = torch.cat([100 * h + torch.arange(keep * hkv * d).reshape(keep, hkv, d)
                         for h in range(4)]).to(torch.bfloat16).float()
