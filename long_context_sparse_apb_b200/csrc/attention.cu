@@ -11,12 +11,17 @@
 // beyond a diagonal are never visited and only the last tile of each range
 // needs a mask.  Every K and V tile in shared memory feeds both query tiles.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3  softmax + epilogue of query tile A (thread r owns row r, which
 //              is TMEM lane r of S_A, P_A and O_A);
 //   warps 4-7  the same for query tile B;
-//   warp 8     TMA producer (Q_A, Q_B once, K and V tiles into 2-stage rings);
-//   warp 9     TMEM allocator and the single UMMA-issuing thread.
+//   warp 8     TMA producer (Q_A, Q_B once, K in a 2-stage and V in a 3-stage
+//              ring);
+//   warp 9     TMEM allocator and the single UMMA-issuing thread, which never
+//              reads shared memory inside its loop;
+//   warp 10    watcher: waits on the barriers the issuer depends on (K, V
+//              landed; each P half written) and hands each one over to the
+//              issuer at a named barrier.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // P_A (bf16, two per 32-bit column) overwrites S_A columns [0,64) once the
 // softmax has read S_A; likewise P_B in S_B.
@@ -45,7 +50,11 @@ namespace apb {
 namespace {
 
 constexpr int kRows = 128;                    // query rows per tile = KV rows per tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
+constexpr int kProducerWarp = 8;
+constexpr int kIssuerWarp = 9;
+constexpr int kWatcherWarp = 10;
+constexpr int kHandoffBar = 1;                // named barrier: watcher -> issuer (64 threads)
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kKStages = 2;
@@ -166,11 +175,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_flags[0] = *gabort;
     s_flags[1] = 0u;
   }
-  if (warp == 9) {
+  if (warp == kIssuerWarp) {
     ptx::tmem_alloc(s_tmem, 512);
     ptx::tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     ptx::tma_prefetch_desc(&mQ);
     ptx::tma_prefetch_desc(&mK);
     ptx::tma_prefetch_desc(&mV);
@@ -188,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK0 = smem + L::kK0;   // stage s at sK0 + s * kTile
   uint8_t* sV0 = smem + L::kV0;
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !skip) {
       int lastK[kKStages], lastV[kVStages];   // last load parity per slot (-1: never loaded)
@@ -228,9 +237,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kVStages; ++s)
         if (lastV[s] >= 0) ptx::mbar_wait_bounded(&bars[V_FULL + s], lastV[s], never, kWaitLimitNs);
     }
-  } else if (warp == 9) {
+  } else if (warp == kIssuerWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !skip) {
+    // Lane 0 issues every UMMA and commit.  The warp never touches shared
+    // memory in the loop: a shared-memory access (an mbarrier check above
+    // all) right after UMMAs holds the issuing thread until they have read
+    // their operands, which lets the tensor core drain at every check.  The
+    // watcher warp makes the checks instead and hands each one over at named
+    // barrier kHandoffBar, which costs the tensor core nothing.  Both warps
+    // walk the same sequence of handoffs, so they stay in step whatever
+    // happens: after a failed wait the watcher goes on handing over at once
+    // (the abort flag is set), and the issuer finishes its loop on stale
+    // operands, whose results are never stored.
+    if (!skip) {
       const uint32_t idesc_s = ptx::idesc_bf16_f32(kRows, kRows, 0);
       const uint32_t idesc_pv = ptx::idesc_bf16_f32(kRows, D, 1);
       // Descriptors of the first K step of every operand buffer; a K step
@@ -241,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV = ptx::sdesc_sw128(ptx::smem_u32(sV0), kRows * 128, 1024);
       constexpr uint32_t kTile16 = L::kTile >> 4;
       const int T[2] = {TA, TB};
+      const bool issuer = lane == 0;
 
       // S_i(jj) = Q_i K(jj)^T into S_i; K(jj) must have landed
       auto issue_s = [&](int i, int jj) {
@@ -253,92 +273,103 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::umma_commit(&bars[S_FULL + i]);
       };
-      auto wait_k = [&](int jj) -> bool {
-        if (!ptx::mbar_spin_bounded(&bars[K_FULL + jj % kKStages], (jj / kKStages) & 1, gabort,
-                                    kWaitLimitNs)) {
-          record_failure(p.status, kWhereKFull + jj % kKStages, jj);
-          return false;
-        }
+      // the watcher's next check has passed
+      auto handoff = [&]() {
+        __syncwarp();
+        ptx::named_barrier_sync(kHandoffBar, 64);
         ptx::tc_fence_after();
-        return true;
       };
 
-      bool ok = ptx::mbar_wait_bounded(&bars[Q_FULL], 0, gabort, kWaitLimitNs);
-      if (!ok) record_failure(p.status, kWhereQ, 0);
-      if (ok) ok = wait_k(0);
-      if (ok) {
+      handoff();                                   // Q_A, Q_B, K(0)
+      if (issuer) {
         issue_s(0, 0);
         if (TB > 0) issue_s(1, 0);
         ptx::umma_commit(&bars[K_EMPTY + 0]);
       }
-      // A thread's shared-memory access (an mbarrier check included) right
-      // after it issued UMMAs waits until they have read their operands, so
-      // every check between two UMMA runs lets the tensor core drain.  The
-      // checks are therefore grouped at the head of each run.
-      for (int j = 0; ok && j < Tmax; ++j) {
+      for (int j = 0; j < Tmax; ++j) {
         const int s = j % kVStages;
-        if (!ptx::mbar_spin_bounded(&bars[V_FULL + s], (j / kVStages) & 1, gabort, kWaitLimitNs)) {
-          record_failure(p.status, kWhereVFull + s, j);
-          break;
-        }
-        // K(j+1), read by this iteration's S MMAs, is checked here with V(j)
         const bool k_next = j + 1 < Tmax;
-        if (k_next && !(ok = wait_k(j + 1))) break;
-        ptx::tc_fence_after();
-        for (int i = 0; i < 2 && ok; ++i) {
+        handoff();                                 // V(j) and K(j+1)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
           if (j >= T[i]) continue;
           const uint32_t tP = tmem + 128 * i;
           const uint32_t tOi = tmem + 256 + 128 * i;
           const uint64_t v = dV + s * kTile16;
-          // P_i(j) arrives in two 64-column halves; PV on the first half may
-          // overlap the softmax's exponentials of the second.  When the second
-          // half is already there both go as one run.
-          if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i], j & 1, gabort, kWaitLimitNs)) {
-            record_failure(p.status, kWhereP + 2 * i, j);
-            ok = false;
-            break;
-          }
           const uint32_t acc0 = j > 0 ? 1u : 0u;
-          if (ptx::mbar_test_wait(ptx::smem_u32(&bars[P_FULL + 2 * i + 1]), j & 1)) {
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              ptx::umma_bf16_ts(tOi, tP + kk * 8, v + ((kk * 2048) >> 4), idesc_pv,
-                                kk > 0 ? 1u : acc0);
-            ptx::umma_commit(&bars[PV0_DONE + i]);
-          } else {
-            ptx::tc_fence_after();
+          // P_i(j) arrives in two 64-column halves; PV on the first half
+          // overlaps the softmax's exponentials of the second
+          handoff();                               // P_i(j), first half
+          if (issuer) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               ptx::umma_bf16_ts(tOi, tP + kk * 8, v + ((kk * 2048) >> 4), idesc_pv,
                                 kk > 0 ? 1u : acc0);
             ptx::umma_commit(&bars[PV0_DONE + i]);
-            if (!ptx::mbar_spin_bounded(&bars[P_FULL + 2 * i + 1], j & 1, gabort,
-                                        kWaitLimitNs)) {
-              record_failure(p.status, kWhereP + 2 * i + 1, j);
-              ok = false;
-              break;
-            }
-            ptx::tc_fence_after();
+          }
+          handoff();                               // P_i(j), second half
+          if (issuer) {
 #pragma unroll
             for (int kk = 4; kk < 8; ++kk)
               ptx::umma_bf16_ts(tOi, tP + kk * 8, v + ((kk * 2048) >> 4), idesc_pv, 1u);
-          }
-          // V(j)'s last reader is PV_B(j) (or PV_A(j) when tile B has no tile j):
-          // release its slot now, before the next S MMA, so its reload starts early
-          if (i == 1 || j >= T[1]) ptx::umma_commit(&bars[V_EMPTY + s]);
-          if (j + 1 < T[i]) {
-            issue_s(i, j + 1);
-          } else {
-            ptx::umma_commit(&bars[O_FINAL + i]);
+            // V(j)'s last reader is PV_B(j) (or PV_A(j) when tile B has no tile
+            // j): release its slot now, before the next S MMA
+            if (i == 1 || j >= T[1]) ptx::umma_commit(&bars[V_EMPTY + s]);
+            if (j + 1 < T[i]) {
+              issue_s(i, j + 1);
+            } else {
+              ptx::umma_commit(&bars[O_FINAL + i]);
+            }
           }
         }
-        if (!ok) break;
-        if (k_next) ptx::umma_commit(&bars[K_EMPTY + (j + 1) % kKStages]);
+        if (issuer && k_next) ptx::umma_commit(&bars[K_EMPTY + (j + 1) % kKStages]);
       }
       // drain every MMA issued so far
-      ptx::umma_commit(&bars[DRAIN]);
-      ptx::mbar_wait_bounded(&bars[DRAIN], 0, never, kWaitLimitNs);
+      if (issuer) {
+        ptx::umma_commit(&bars[DRAIN]);
+        ptx::mbar_wait_bounded(&bars[DRAIN], 0, never, kWaitLimitNs);
+      }
+    }
+  } else if (warp == kWatcherWarp) {
+    // ------------------------------------------------------------ watcher
+    // Makes the issuer's barrier checks, in the issuer's order, and hands
+    // each one over at kHandoffBar.  After a failed wait (recorded, abort flag
+    // set) the remaining waits return at once, so the hand-overs continue and
+    // the issuer is never left waiting.
+    if (!skip) {
+      const int T[2] = {TA, TB};
+      bool ok = true;
+      auto check = [&](uint64_t* bar, uint32_t parity, uint32_t where, int tile) {
+        bool got = true;
+        if (lane == 0) {
+          got = ptx::mbar_wait_bounded(bar, parity, gabort, kWaitLimitNs);
+          if (!got && ok) record_failure(p.status, where, tile);
+        }
+        ok = __shfl_sync(0xffffffffu, (int)(got && ok), 0) != 0;
+      };
+      auto handoff = [&]() {
+        __syncwarp();
+        ptx::named_barrier_sync(kHandoffBar, 64);
+      };
+      check(&bars[Q_FULL], 0, kWhereQ, 0);
+      check(&bars[K_FULL], 0, kWhereKFull, 0);
+      handoff();
+      for (int j = 0; j < Tmax; ++j) {
+        const int s = j % kVStages;
+        check(&bars[V_FULL + s], (j / kVStages) & 1, kWhereVFull + s, j);
+        if (j + 1 < Tmax)
+          check(&bars[K_FULL + (j + 1) % kKStages], ((j + 1) / kKStages) & 1,
+                kWhereKFull + (j + 1) % kKStages, j + 1);
+        handoff();
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (j >= T[i]) continue;
+          check(&bars[P_FULL + 2 * i], j & 1, kWhereP + 2 * i, j);
+          handoff();
+          check(&bars[P_FULL + 2 * i + 1], j & 1, kWhereP + 2 * i + 1, j);
+          handoff();
+        }
+      }
     }
   } else if (!skip) {
     // ------------------------------------------------------------ softmax
@@ -548,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kIssuerWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
   }
