@@ -19,9 +19,10 @@
 //              ring);
 //   warp 9     TMEM allocator and the single UMMA-issuing thread, which never
 //              reads shared memory inside its loop;
-//   warp 10    watcher: waits on the barriers the issuer depends on (K, V
-//              landed; each P half written) and hands each one over to the
-//              issuer at a named barrier.
+//   warp 10    watcher: waits on the TMA barriers the issuer depends on (Q, K,
+//              V landed) and hands each one over to the issuer at a named
+//              barrier; the softmax warps hand each P half over themselves,
+//              at named barriers of their own.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // P_A (bf16, two per 32-bit column) overwrites S_A columns [0,64) once the
 // softmax has read S_A; likewise P_B in S_B.
@@ -29,7 +30,8 @@
 //   S_i(j) = Q_i K(j)^T         tcgen05.mma, A and B from shared memory
 //   softmax_i reads S_i(j), exponentiates against a lazily moved row maximum
 //   (O_i is rescaled in TMEM only when that base moves), writes P_i(j) to
-//   TMEM in two 64-column halves, signals P_FULL_i per half
+//   TMEM in two 64-column halves and hands each half to the issuer at a
+//   named barrier
 //   O_i += P_i(j) V(j)          tcgen05.mma, A = P_i from TMEM, B = V
 // The MMA thread issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while one
 // softmax warpgroup works on its tile the tensor core serves the other.
@@ -55,6 +57,10 @@ constexpr int kProducerWarp = 8;
 constexpr int kIssuerWarp = 9;
 constexpr int kWatcherWarp = 10;
 constexpr int kHandoffBar = 1;                // named barrier: watcher -> issuer (64 threads)
+// Named barriers 2..5: P_i(j) half h written -> issuer, id kPBar + 2 * i + h;
+// the 128 softmax threads of tile i arrive, the issuer warp waits.
+constexpr int kPBar = 2;
+constexpr int kPBarThreads = 128 + 32;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kKStages = 2;
@@ -69,7 +75,6 @@ constexpr uint32_t kWhereKFull = 51;    // issuer, + K slot
 constexpr uint32_t kWhereVFull = 54;    // issuer, + V slot
 constexpr uint32_t kWhereS = 60;        // softmax, + query tile
 constexpr uint32_t kWhereO = 63;        // epilogue, + query tile
-constexpr uint32_t kWhereP = 70;        // issuer, + 2 * query tile + half
 constexpr uint32_t kWherePV0 = 74;      // softmax, + query tile (rare rescale path)
 
 enum Bar {
@@ -79,8 +84,7 @@ enum Bar {
   V_FULL = K_EMPTY + kKStages,      // kVStages
   V_EMPTY = V_FULL + kVStages,      // kVStages
   S_FULL = V_EMPTY + kVStages,      // per query tile (A, B)
-  P_FULL = S_FULL + 2,              // per query tile and 64-column half: + 2 * tile + half
-  O_FINAL = P_FULL + 4,             // per query tile
+  O_FINAL = S_FULL + 2,             // per query tile
   DRAIN = O_FINAL + 2,
   PV0_DONE = DRAIN + 1,             // per query tile: PV_i(j) on the first P half has run
   NUM_BARS = PV0_DONE + 2
@@ -170,7 +174,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM_BARS; ++i) ptx::mbar_init(&bars[i], 1);
-    for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars[P_FULL + i], 128);
     ptx::fence_mbar_init();
     s_flags[0] = *gabort;
     s_flags[1] = 0u;
@@ -243,12 +246,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // memory in the loop: a shared-memory access (an mbarrier check above
     // all) right after UMMAs holds the issuing thread until they have read
     // their operands, which lets the tensor core drain at every check.  The
-    // watcher warp makes the checks instead and hands each one over at named
-    // barrier kHandoffBar, which costs the tensor core nothing.  Both warps
-    // walk the same sequence of handoffs, so they stay in step whatever
-    // happens: after a failed wait the watcher goes on handing over at once
-    // (the abort flag is set), and the issuer finishes its loop on stale
-    // operands, whose results are never stored.
+    // TMA checks are made by the watcher warp and handed over at named
+    // barrier kHandoffBar; each half of P_i is handed over by tile i's
+    // softmax threads at named barrier kPBar + 2i + h (they arrive, the
+    // issuer waits).  A named barrier costs the tensor core nothing.  Every
+    // party walks the same sequence of handoffs, so they stay in step
+    // whatever happens: after a failed wait the watcher goes on handing over
+    // at once (the abort flag is set), a softmax warp that gave up meets the
+    // issuer at each remaining P barrier, and the issuer finishes its loop on
+    // stale operands, whose results are never stored.
     if (!skip) {
       const uint32_t idesc_s = ptx::idesc_bf16_f32(kRows, kRows, 0);
       const uint32_t idesc_pv = ptx::idesc_bf16_f32(kRows, D, 1);
@@ -279,6 +285,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::named_barrier_sync(kHandoffBar, 64);
         ptx::tc_fence_after();
       };
+      // the softmax threads of tile i have written half h of P_i
+      auto p_ready = [&](int i, int h) {
+        __syncwarp();
+        ptx::named_barrier_sync(kPBar + 2 * i + h, kPBarThreads);
+        ptx::tc_fence_after();
+      };
 
       handoff();                                   // Q_A, Q_B, K(0)
       if (issuer) {
@@ -299,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t acc0 = j > 0 ? 1u : 0u;
           // P_i(j) arrives in two 64-column halves; PV on the first half
           // overlaps the softmax's exponentials of the second
-          handoff();                               // P_i(j), first half
+          p_ready(i, 0);
           if (issuer) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -307,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 kk > 0 ? 1u : acc0);
             ptx::umma_commit(&bars[PV0_DONE + i]);
           }
-          handoff();                               // P_i(j), second half
+          p_ready(i, 1);
           if (issuer) {
 #pragma unroll
             for (int kk = 4; kk < 8; ++kk)
@@ -332,17 +344,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWatcherWarp) {
     // ------------------------------------------------------------ watcher
-    // Makes the issuer's barrier checks, in the issuer's order, and hands
-    // each one over at kHandoffBar.  After a failed wait (recorded, abort flag
-    // set) the remaining waits return at once, so the hand-overs continue and
-    // the issuer is never left waiting.
+    // Makes the issuer's checks of the TMA loads (Q, K(j+1) with V(j)), in
+    // the issuer's order, and hands each one over at kHandoffBar.  After a
+    // failed wait (recorded, abort flag set) the remaining waits return at
+    // once, so the hand-overs continue and the issuer is never left waiting.
     if (!skip) {
-      const int T[2] = {TA, TB};
       bool ok = true;
       auto check = [&](uint64_t* bar, uint32_t parity, uint32_t where, int tile) {
         bool got = true;
         if (lane == 0) {
-          got = ptx::mbar_wait_bounded(bar, parity, gabort, kWaitLimitNs);
+          // polled: this warp's reaction time is on the issuer's path
+          got = ptx::mbar_spin_bounded(bar, parity, gabort, kWaitLimitNs);
           if (!got && ok) record_failure(p.status, where, tile);
         }
         ok = __shfl_sync(0xffffffffu, (int)(got && ok), 0) != 0;
@@ -361,14 +373,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           check(&bars[K_FULL + (j + 1) % kKStages], ((j + 1) / kKStages) & 1,
                 kWhereKFull + (j + 1) % kKStages, j + 1);
         handoff();
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if (j >= T[i]) continue;
-          check(&bars[P_FULL + 2 * i], j & 1, kWhereP + 2 * i, j);
-          handoff();
-          check(&bars[P_FULL + 2 * i + 1], j & 1, kWhereP + 2 * i + 1, j);
-          handoff();
-        }
       }
     }
   } else if (!skip) {
@@ -382,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q0 = qA0 + i * kRows;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    int arrived = 0;   // P halves handed to the issuer so far (2 per KV tile)
     for (int j = 0; j < T; ++j) {
       ok = ptx::mbar_wait_bounded(&bars[S_FULL + i], j & 1, gabort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -493,7 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       APB_TMEM_ST32(tS, pk);
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars[P_FULL + 2 * i]);
+      ptx::named_barrier_arrive(kPBar + 2 * i, kPBarThreads);
+      ++arrived;
       // ---- second half
       APB_TMEM_LD64(tS + 64, sr);
       if (lim < kRows) {
@@ -538,10 +544,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       APB_TMEM_ST32(tS + 32, pk);
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars[P_FULL + 2 * i + 1]);
+      ptx::named_barrier_arrive(kPBar + 2 * i + 1, kPBarThreads);
+      ++arrived;
 #pragma unroll
       for (int x = 0; x < 4; ++x) sum[x] += sum1[x];
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+    }
+    if (!ok) {
+      // The issuer waits for every P half of this tile at named barriers,
+      // which have no time limit: meet it at each remaining one (blocking,
+      // so that this warp never runs a phase ahead of it).
+      for (int a = arrived; a < 2 * T; ++a) {
+        __syncwarp();
+        ptx::named_barrier_sync(kPBar + 2 * i + (a & 1), kPBarThreads);
+      }
     }
     if (ok && T > 0) {
       ok = ptx::mbar_wait_bounded(&bars[O_FINAL + i], 0, gabort, kWaitLimitNs);
