@@ -431,7 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto check = [&](int bar, uint32_t parity, uint32_t where, int tile) {
         bool got = true;
         if (lane == 0) {
-          got = pair::wait_cluster_bounded(&bars[bar], parity, gabort, kWaitLimitNs);
+          // polled: this warp's reaction time is on the issuer's path
+          got = pair::spin_cluster_bounded(&bars[bar], parity, gabort, kWaitLimitNs);
           if (!got && ok) record_failure(p.status, where, tile);
         }
         ok = __shfl_sync(0xffffffffu, (int)(got && ok), 0) != 0;
