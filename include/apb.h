@@ -289,6 +289,19 @@ apb_status apb_score_compress_static_selftest(uint32_t limit_us, void* stream);
 apb_status apb_selftest_wait_timeout(void* workspace, size_t ws_bytes, uint32_t limit_us,
                                      void* stream);
 
+/* No counterpart in the paper: failure-path self-test.  Launches one thread
+ * on `stream` that waits delay_us microseconds (<= 1000000) and then sets
+ * the launch-wide abort flag in the status block of `workspace` (>= 256
+ * bytes), exactly as a kernel whose bounded wait ran out does.  Launched on
+ * a second stream while a score or attention kernel runs on the same
+ * workspace, it makes that kernel's waits give up mid-run: the kernel must
+ * still finish (every CTA drains its copies and MMAs and meets its partner
+ * warps at each remaining named barrier), and apb_device_status then reports
+ * APB_ERR_TIMEOUT.  Outputs of the aborted call are undefined.  Nothing
+ * faults, traps or hangs. */
+apb_status apb_selftest_abort_after(void* workspace, size_t ws_bytes, uint32_t delay_us,
+                                    void* stream);
+
 /* Synchronises `stream`, then reads the status block of `workspace`:
  * APB_ERR_TIMEOUT if a kernel recorded a bounded wait that ran out since the
  * block was last cleared, else APB_OK (APB_ERR_CUDA if the reads fail).

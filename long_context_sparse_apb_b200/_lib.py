@@ -67,6 +67,8 @@ _lib.apb_score_compress_static_status.argtypes = [_P, ctypes.c_int]
 _lib.apb_score_compress_static_status.restype = ctypes.c_int
 _lib.apb_score_compress_static_selftest.argtypes = [ctypes.c_uint32, _P]
 _lib.apb_score_compress_static_selftest.restype = ctypes.c_int
+_lib.apb_selftest_abort_after.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
+_lib.apb_selftest_abort_after.restype = ctypes.c_int
 _lib.apb_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
 _lib.apb_selftest_wait_timeout.restype = ctypes.c_int
 _lib.apb_device_status.argtypes = [_P, _P, ctypes.c_int]
@@ -435,6 +437,14 @@ def selftest_wait_timeout(workspace, limit_us: int, stream=None):
     st = _lib.apb_selftest_wait_timeout(_ptr(workspace), workspace.numel(), limit_us,
                                         _stream(stream))
     _check(st, "apb_selftest_wait_timeout")
+
+
+def selftest_abort_after(workspace, delay_us: int, stream=None):
+    """apb_selftest_abort_after: sets the workspace's abort flag after
+    delay_us from a one-thread kernel on `stream`."""
+    st = _lib.apb_selftest_abort_after(_ptr(workspace), workspace.numel(), delay_us,
+                                       _stream(stream))
+    _check(st, "apb_selftest_abort_after")
 
 
 class Prefill:
