@@ -32,9 +32,6 @@
 //              fp32 and write qh, ql (2-pair ring) in the 128-byte-swizzled
 //              K-major layout UMMA reads;
 //   warp 13    UMMA issuer (even CTA) / TMEM allocation (both);
-//   warp 15    watcher (even CTA): waits on the barriers the issuer depends on
-//              and hands each one over to it at a named barrier, so that the
-//              issuer never touches shared memory between UMMA runs;
 //   warps 0-3  epilogue, one token row per thread.
 // Full barriers live in the even CTA and count both CTAs' arrivals; empty
 // barriers live in both and get one commit each.  Waits are bounded like the
@@ -72,9 +69,7 @@ constexpr int kConvThreads = 256;          // warps 4-11
 constexpr int kBWarp = 12;
 constexpr int kMmaWarp = 13;
 constexpr int kKVWarp = 14;
-constexpr int kWatchWarp = 15;
-constexpr int kThreads = 512;
-constexpr int kHandoffBar = 3;             // named barrier: watcher -> issuer (even CTA)
+constexpr int kThreads = 480;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
 
@@ -239,7 +234,7 @@ __device__ __forceinline__ void q_split_store(const QAcc& A, float invG, int sp,
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(512, 1)   // 512: caps registers at 128 (launched with 480)
     score_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                  const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mW,
                  const ScoreParams p) {
@@ -345,17 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ UMMA issuer
-    // Lane 0 of the even CTA issues every pair UMMA and commit.  The warp
-    // reads no shared memory inside its loop (a shared-memory access right
-    // after UMMAs holds the issuing thread until they have read their
-    // operands, letting the tensor core drain at every check): the watcher
-    // warp makes the barrier checks in the issuer's order and hands each one
-    // over at named barrier kHandoffBar.  After a failed wait the watcher
-    // keeps handing over at once (abort flag set), so both finish their
-    // loops; results of a failed launch are never trusted (the status block
-    // reports it).
-    if (rank == 0 && !skip) {
-      const bool issuer = lane == 0;
+    if (lane == 0 && rank == 0 && !skip) {
       const uint32_t idesc = ptx::idesc_bf16_f32(2 * kTile, kHid, 0);
       const uint32_t aKV = ptx::smem_u32(smem + kSmemKV);
       const uint32_t aQ = ptx::smem_u32(smem + kSmemQ);
@@ -365,29 +350,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         pair::umma_commit(pair::map_to(&bars[bar], 0));
         pair::umma_commit(pair::map_to(&bars[bar], 1));
       };
-      auto handoff = [&]() {
-        __syncwarp();
-        ptx::named_barrier_sync(kHandoffBar, 64);
-        ptx::tc_fence_after();
-      };
       int kvu = 0, qu = 0, bu = 0, it = 0;
-      for (int t = cl; t < p.n_tiles; t += ncl, ++it) {
+      bool ok = true;
+      for (int t = cl; t < p.n_tiles && ok; t += ncl, ++it) {
         const int b = it & 1;
-        handoff();                                     // accumulator b free
+        if (!pair::spin_cluster_bounded(&bars[ACC_EMPTY + b], ((it >> 1) & 1) ^ 1, gabort,
+                                        kWaitLimitNs)) {
+          record_failure(p.status, 84, it);
+          break;
+        }
+        ptx::tc_fence_after();
         const uint32_t acc = tmem + 256 * b;
-        for (int i = 0; i < p.n_chunks; ++i) {
+        bool first = true;
+        for (int i = 0; i < p.n_chunks && ok; ++i) {
           const int c = chunk_at(i);
           const int bs = bu % kBStages;
           const bool qsec = chunk_section(c, p.d) == 2;
           const int s = qsec ? qu % kQStages : kvu % kKVStages;
-          handoff();                                   // weights and x of chunk c
+          ok = pair::spin_cluster_bounded(&bars[B_FULL + bs], (bu / kBStages) & 1, gabort,
+                                          kWaitLimitNs) &&
+               (qsec ? pair::spin_cluster_bounded(&bars[Q_FULL + s], (qu / kQStages) & 1, gabort,
+                                                  kWaitLimitNs)
+                     : pair::spin_cluster_bounded(&bars[KV_FULL + s], (kvu / kKVStages) & 1,
+                                                  gabort, kWaitLimitNs));
+          if (!ok) {
+            record_failure(p.status, 85, c);
+            break;
+          }
+          ptx::tc_fence_after();
           const uint32_t bh = aB + bs * 2 * kBPart, bl = bh + kBPart;
           const uint32_t xh = qsec ? aQ + s * 2 * kATile : aKV + s * kATile;
           const uint32_t xl = xh + kATile;     // ql (q chunks only)
-          const uint32_t acc0 = i == 0 ? 0u : 1u;
+          const uint32_t acc0 = first ? 0u : 1u;
+          first = false;
           // the two forms as separate straight-line runs: a branch between
           // consecutive UMMAs slows the tensor core's stream (~1.6x here)
-          if (issuer && qsec) {
+          if (qsec) {
 #pragma unroll
             for (int ks = 0; ks < kChunk / 16; ++ks) {
               const uint64_t dXh = ptx::sdesc_sw128(xh + ks * 32, 16, 1024);
@@ -398,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               pair::umma_bf16_ss(acc, dXh, dBl, idesc, 1u);
               pair::umma_bf16_ss(acc, dXl, dBh, idesc, 1u);
             }
-          } else if (issuer) {
+          } else {
 #pragma unroll
             for (int ks = 0; ks < kChunk / 16; ++ks) {
               const uint64_t dXh = ptx::sdesc_sw128(xh + ks * 32, 16, 1024);
@@ -408,58 +406,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               pair::umma_bf16_ss(acc, dXh, dBl, idesc, 1u);
             }
           }
-          if (issuer) {
-            commit_both(qsec ? Q_EMPTY + s : KV_EMPTY + s);
-            commit_both(B_EMPTY + bs);
-          }
+          commit_both(qsec ? Q_EMPTY + s : KV_EMPTY + s);
+          commit_both(B_EMPTY + bs);
           ++bu;
           if (qsec) ++qu; else ++kvu;
         }
-        if (issuer) commit_both(ACC_FULL + b);
+        if (ok) commit_both(ACC_FULL + b);
       }
-      if (issuer) {
-        commit_both(DRAIN);
-        ptx::mbar_wait_bounded(&bars[DRAIN], 0, never, kWaitLimitNs);
-      }
-    }
-  } else if (warp == kWatchWarp) {
-    // ------------------------------------------------------------ watcher
-    // The issuer's barrier checks, in its order, each handed over at
-    // kHandoffBar (even CTA only).
-    if (rank == 0 && !skip) {
-      bool ok = true;
-      auto check = [&](int bar, uint32_t parity, uint32_t where, int tile) {
-        bool got = true;
-        if (lane == 0) {
-          // polled: this warp's reaction time is on the issuer's path
-          got = pair::spin_cluster_bounded(&bars[bar], parity, gabort, kWaitLimitNs);
-          if (!got && ok) record_failure(p.status, where, tile);
-        }
-        ok = __shfl_sync(0xffffffffu, (int)(got && ok), 0) != 0;
-      };
-      auto handoff = [&]() {
-        __syncwarp();
-        ptx::named_barrier_sync(kHandoffBar, 64);
-      };
-      int kvu = 0, qu = 0, bu = 0, it = 0;
-      for (int t = cl; t < p.n_tiles; t += ncl, ++it) {
-        const int b = it & 1;
-        check(ACC_EMPTY + b, ((it >> 1) & 1) ^ 1, 84, it);
-        handoff();
-        for (int i = 0; i < p.n_chunks; ++i) {
-          const int c = chunk_at(i);
-          const int bs = bu % kBStages;
-          const bool qsec = chunk_section(c, p.d) == 2;
-          check(B_FULL + bs, (bu / kBStages) & 1, 85, c);
-          if (qsec)
-            check(Q_FULL + qu % kQStages, (qu / kQStages) & 1, 85, c);
-          else
-            check(KV_FULL + kvu % kKVStages, (kvu / kKVStages) & 1, 85, c);
-          handoff();
-          ++bu;
-          if (qsec) ++qu; else ++kvu;
-        }
-      }
+      commit_both(DRAIN);
+      ptx::mbar_wait_bounded(&bars[DRAIN], 0, never, kWaitLimitNs);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ q converters
