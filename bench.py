@@ -233,17 +233,25 @@ def run_reference(args, cfg):
         return
     x = inputs.generate(cfg)
     rows = args.oracle_rows
-    vals = []
+    vals, secs = [], []
     for i in range(args.warmup + args.steps):
-        v, _ = oracle_sample(cfg, x, rows)
+        v, meas = oracle_sample(cfg, x, rows)
         if i >= args.warmup:
             vals.append(v)
+            secs.append(meas)
     value = statistics.median(vals)
+    # one step = one bounded sample, timed as it ran; `value` is the tokens of
+    # the whole sequence over the sample's time extrapolated to the sequence,
+    # so a step stands for value * step-seconds tokens of work
+    ms_per_step = statistics.median(secs) * 1e3
     sample = (f"per step: scoring+top-k of host 0 (x{cfg.n_hosts} hosts), passing block of every "
               f"host, attention of {rows} rows/host on all {cfg.n_q_heads} q heads "
-              f"(x{cfg.block_len // rows}); NumPy float64")
+              f"(x{cfg.block_len // rows}); NumPy float64; a step is this sample "
+              f"({ms_per_step / 1e3:.1f} s measured), worth {value * ms_per_step / 1e3:.0f} of "
+              f"the sequence's {cfg.seq_len} tokens at the extrapolated rate")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": cfg.seq_len / value * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "tokens_equiv_per_step": value * ms_per_step / 1e3,
             "higher_is_better": True, "scaling": "weak" if args.mode == "replicas" else "strong",
             "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_dict(cfg, args.gpus, args.mode),

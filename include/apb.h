@@ -289,18 +289,18 @@ apb_status apb_score_compress_static_selftest(uint32_t limit_us, void* stream);
 apb_status apb_selftest_wait_timeout(void* workspace, size_t ws_bytes, uint32_t limit_us,
                                      void* stream);
 
-/* No counterpart in the paper: failure-path self-test.  Launches one thread
- * on `stream` that waits delay_us microseconds (<= 1000000) and then sets
- * the launch-wide abort flag in the status block of `workspace` (>= 256
- * bytes), exactly as a kernel whose bounded wait ran out does.  Launched on
- * a second stream while a score or attention kernel runs on the same
- * workspace, it makes that kernel's waits give up mid-run: the kernel must
- * still finish (every CTA drains its copies and MMAs and meets its partner
- * warps at each remaining named barrier), and apb_device_status then reports
- * APB_ERR_TIMEOUT.  Outputs of the aborted call are undefined.  Nothing
- * faults, traps or hangs. */
-apb_status apb_selftest_abort_after(void* workspace, size_t ws_bytes, uint32_t delay_us,
-                                    void* stream);
+/* No counterpart in the paper: failure-path self-test.  Sets the time limit
+ * of the bounded on-chip waits of every kernel launched afterwards by this
+ * process (default 1 s; limit_ns = 0 restores it; otherwise limit_ns must be
+ * >= 100).  A wait gives up only after its barrier has failed 32 or more
+ * polls and the limit has passed, so a short limit makes the waits that
+ * really block (on the tensor core, the copies, the other warps) run out
+ * mid-run: every kernel must still finish (each CTA drains its copies and
+ * MMAs and meets its partner warps at every remaining named barrier) and
+ * apb_device_status then reports APB_ERR_TIMEOUT; the outputs of such a call
+ * are undefined.  Process-wide, not thread-safe against concurrent launches;
+ * meant for tests.  Nothing faults, traps or hangs. */
+apb_status apb_selftest_set_wait_limit(uint64_t limit_ns);
 
 /* Synchronises `stream`, then reads the status block of `workspace`:
  * APB_ERR_TIMEOUT if a kernel recorded a bounded wait that ran out since the

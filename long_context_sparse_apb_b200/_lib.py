@@ -67,8 +67,8 @@ _lib.apb_score_compress_static_status.argtypes = [_P, ctypes.c_int]
 _lib.apb_score_compress_static_status.restype = ctypes.c_int
 _lib.apb_score_compress_static_selftest.argtypes = [ctypes.c_uint32, _P]
 _lib.apb_score_compress_static_selftest.restype = ctypes.c_int
-_lib.apb_selftest_abort_after.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
-_lib.apb_selftest_abort_after.restype = ctypes.c_int
+_lib.apb_selftest_set_wait_limit.argtypes = [ctypes.c_uint64]
+_lib.apb_selftest_set_wait_limit.restype = ctypes.c_int
 _lib.apb_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
 _lib.apb_selftest_wait_timeout.restype = ctypes.c_int
 _lib.apb_device_status.argtypes = [_P, _P, ctypes.c_int]
@@ -439,12 +439,10 @@ def selftest_wait_timeout(workspace, limit_us: int, stream=None):
     _check(st, "apb_selftest_wait_timeout")
 
 
-def selftest_abort_after(workspace, delay_us: int, stream=None):
-    """apb_selftest_abort_after: sets the workspace's abort flag after
-    delay_us from a one-thread kernel on `stream`."""
-    st = _lib.apb_selftest_abort_after(_ptr(workspace), workspace.numel(), delay_us,
-                                       _stream(stream))
-    _check(st, "apb_selftest_abort_after")
+def selftest_set_wait_limit(limit_ns: int):
+    """apb_selftest_set_wait_limit: time limit of the kernels' bounded waits
+    for later launches (0 restores the default 1 s)."""
+    _check(_lib.apb_selftest_set_wait_limit(limit_ns), "apb_selftest_set_wait_limit")
 
 
 class Prefill:

@@ -1,6 +1,7 @@
 // C-ABI layer: argument checks, workspace layout, status reporting.
 // Every entry point validates on the host before launching anything and
 // returns an apb_status; no exception or abort crosses the boundary.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -10,6 +11,8 @@
 
 namespace {
 thread_local char g_last_error[512] = "";
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;   // 1 s
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 }  // namespace
 
 namespace apb {
@@ -25,6 +28,8 @@ apb_status fail(apb_status st, const char* fmt, ...) {
 apb_status cuda_fail(cudaError_t e, const char* what) {
   return fail(APB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
+
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 }  // namespace apb
 
@@ -380,5 +385,13 @@ const char* apb_status_string(apb_status status) {
 }
 
 const char* apb_last_error(void) { return g_last_error; }
+
+apb_status apb_selftest_set_wait_limit(uint64_t limit_ns) {
+  if (limit_ns != 0 && limit_ns < 100)
+    return fail(APB_ERR_INVALID_ARG, "apb_selftest_set_wait_limit: limit_ns=%llu < 100",
+                (unsigned long long)limit_ns);
+  g_wait_ns.store(limit_ns == 0 ? kDefaultWaitNs : limit_ns, std::memory_order_relaxed);
+  return APB_OK;
+}
 
 }  // extern "C"

@@ -15,6 +15,10 @@ namespace apb {
 apb_status fail(apb_status st, const char* fmt, ...);
 apb_status cuda_fail(cudaError_t e, const char* what);
 
+// Time limit of the kernels' bounded waits for launches made now (1 s
+// unless a test shortened it with apb_selftest_set_wait_limit).
+uint64_t wait_limit_ns();
+
 // Status block at the start of every workspace.
 // "where" codes: 40-75 the attention kernel (named kWhere* in
 // attention.cu), 80-90 the score kernel (80/82 + CTA rank: weight / k,v

@@ -61,7 +61,7 @@ constexpr int kHandoffBar = 1;                // named barrier: watcher -> issue
 // the 128 softmax threads of tile i arrive, the issuer warp waits.
 constexpr int kPBar = 2;
 constexpr int kPBarThreads = 128 + 32;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: drains of copies and MMAs
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kKStages = 2;
 constexpr int kVStages = 3;   // V is released later than K: one more stage of prefetch
@@ -111,6 +111,7 @@ struct Params {
   int h0, hcount, hstride, q_row0, k_row0, anchor_row0;
   long long N;   // rows of the Q/out buffer (the lse row stride)
   float scale_log2;
+  uint64_t wait_ns;   // limit of the bounded waits (1 s; shorter in self-tests)
   __nv_bfloat16* out;
   float* lse;
   DeviceStatus* status;
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < Tmax; ++j) {
         const int ks = j % kKStages, vs = j % kVStages;
         const uint32_t kpar = (j / kKStages) & 1, vpar = (j / kVStages) & 1;
-        if (!ptx::mbar_wait_bounded(&bars[K_EMPTY + ks], kpar ^ 1, gabort, kWaitLimitNs)) {
+        if (!ptx::mbar_wait_bounded(&bars[K_EMPTY + ks], kpar ^ 1, gabort, p.wait_ns)) {
           record_failure(p.status, kWhereKEmpty + ks, j);
           break;
         }
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         load_kv_tile<D>(&mK, &mPK, sK0 + ks * L::kTile, &bars[K_FULL + ks], j, na, np, g,
                         local_row0, p.anchor_row0);
         lastK[ks] = (int)kpar;
-        if (!ptx::mbar_wait_bounded(&bars[V_EMPTY + vs], vpar ^ 1, gabort, kWaitLimitNs)) {
+        if (!ptx::mbar_wait_bounded(&bars[V_EMPTY + vs], vpar ^ 1, gabort, p.wait_ns)) {
           record_failure(p.status, kWhereVEmpty + vs, j);
           break;
         }
@@ -354,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool got = true;
         if (lane == 0) {
           // polled: this warp's reaction time is on the issuer's path
-          got = ptx::mbar_spin_bounded(bar, parity, gabort, kWaitLimitNs);
+          got = ptx::mbar_spin_bounded(bar, parity, gabort, p.wait_ns);
           if (!got && ok) record_failure(p.status, where, tile);
         }
         ok = __shfl_sync(0xffffffffu, (int)(got && ok), 0) != 0;
@@ -388,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int arrived = 0;   // P halves handed to the issuer so far (2 per KV tile)
     for (int j = 0; j < T; ++j) {
-      ok = ptx::mbar_wait_bounded(&bars[S_FULL + i], j & 1, gabort, kWaitLimitNs);
+      ok = ptx::mbar_wait_bounded(&bars[S_FULL + i], j & 1, gabort, p.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) record_failure(p.status, kWhereS + i, j);
         ok = false;
@@ -514,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // rare: m moves after the first half's probabilities went out, so O
         // (which PV_i(j) on the first half is adding to) is rescaled once that
         // PV has run, before the second half's
-        const bool w = ptx::mbar_wait_bounded(&bars[PV0_DONE + i], j & 1, gabort, kWaitLimitNs);
+        const bool w = ptx::mbar_wait_bounded(&bars[PV0_DONE + i], j & 1, gabort, p.wait_ns);
         if (!__all_sync(0xffffffffu, w)) {
           if (lane == 0) record_failure(p.status, kWherePV0 + i, j);
           ok = false;
@@ -560,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (ok && T > 0) {
-      ok = ptx::mbar_wait_bounded(&bars[O_FINAL + i], 0, gabort, kWaitLimitNs);
+      ok = ptx::mbar_wait_bounded(&bars[O_FINAL + i], 0, gabort, p.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) record_failure(p.status, kWhereO + i, T);
         ok = false;
@@ -647,6 +648,7 @@ cudaError_t launch_d(const Shape& s, const HostRange& r, const void* q, const vo
   p.anchor_row0 = r.anchor_row0;
   p.N = r.q_rows;
   p.scale_log2 = s.scale * kLog2e;
+  p.wait_ns = wait_limit_ns();
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.status = status;

@@ -70,7 +70,7 @@ constexpr int kBWarp = 12;
 constexpr int kMmaWarp = 13;
 constexpr int kKVWarp = 14;
 constexpr int kThreads = 480;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // drains at the end of a launch
 constexpr uint64_t kDrainLimitNs = 100000000ull;
 
 // Full barriers (KV_FULL, Q_FULL, B_FULL) and ACC_EMPTY are used in the even
@@ -146,6 +146,7 @@ struct ScoreParams {
   const float* b2;
   float* scores;
   DeviceStatus* status;
+  uint64_t wait_ns;   // limit of the bounded waits (1 s; shorter in self-tests)
 };
 
 // Section of feature chunk c: 0 k, 1 v, 2 q.
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(512, 1)   // 512: caps registers at 128 (launc
           const int sec = chunk_section(c, p.d);
           if (!isB && sec == 2) continue;       // q tiles come from the converters
           const int s = u % stages;
-          if (!ptx::mbar_wait_bounded(&empty[s], ((u / stages) & 1) ^ 1, gabort, kWaitLimitNs)) {
+          if (!ptx::mbar_wait_bounded(&empty[s], ((u / stages) & 1) ^ 1, gabort, p.wait_ns)) {
             record_failure(p.status, (isB ? 80 : 82) + rank, u);
             ok = false;
             break;
@@ -355,7 +356,7 @@ __global__ void __launch_bounds__(512, 1)   // 512: caps registers at 128 (launc
       for (int t = cl; t < p.n_tiles && ok; t += ncl, ++it) {
         const int b = it & 1;
         if (!pair::spin_cluster_bounded(&bars[ACC_EMPTY + b], ((it >> 1) & 1) ^ 1, gabort,
-                                        kWaitLimitNs)) {
+                                        p.wait_ns)) {
           record_failure(p.status, 84, it);
           break;
         }
@@ -368,11 +369,11 @@ __global__ void __launch_bounds__(512, 1)   // 512: caps registers at 128 (launc
           const bool qsec = chunk_section(c, p.d) == 2;
           const int s = qsec ? qu % kQStages : kvu % kKVStages;
           ok = pair::spin_cluster_bounded(&bars[B_FULL + bs], (bu / kBStages) & 1, gabort,
-                                          kWaitLimitNs) &&
+                                          p.wait_ns) &&
                (qsec ? pair::spin_cluster_bounded(&bars[Q_FULL + s], (qu / kQStages) & 1, gabort,
-                                                  kWaitLimitNs)
+                                                  p.wait_ns)
                      : pair::spin_cluster_bounded(&bars[KV_FULL + s], (kvu / kKVStages) & 1,
-                                                  gabort, kWaitLimitNs));
+                                                  gabort, p.wait_ns));
           if (!ok) {
             record_failure(p.status, 85, c);
             break;
@@ -455,7 +456,7 @@ __global__ void __launch_bounds__(512, 1)   // 512: caps registers at 128 (launc
             for (int c = 0; c < n_q && ok; ++c) {
               const int u = qu + c;
               ok = ptx::mbar_wait_bounded(&bars[Q_EMPTY + u % kQStages],
-                                          ((u / kQStages) & 1) ^ 1, gabort, kWaitLimitNs);
+                                          ((u / kQStages) & 1) ^ 1, gabort, p.wait_ns);
               if (!ok) record_failure(p.status, 86 + rank, u);
             }
           ok = ptx::barrier_and(1, kConvThreads, ok);
@@ -493,7 +494,7 @@ __global__ void __launch_bounds__(512, 1)   // 512: caps registers at 128 (launc
         const float4* b1 = reinterpret_cast<const float4*>(s_b1);
         const float4* w2 = reinterpret_cast<const float4*>(s_w2);
         const bool ok = ptx::mbar_wait_bounded(&bars[ACC_FULL + b], (it >> 1) & 1, gabort,
-                                               kWaitLimitNs);
+                                               p.wait_ns);
         if (!ptx::barrier_and(2, kEpiThreads, ok)) {
           if (row == 0) record_failure(p.status, 88 + rank, it);
           break;
@@ -605,6 +606,7 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* k, const voi
   p.b2 = b2;
   p.scores = scores;
   p.status = status;
+  p.wait_ns = wait_limit_ns();
   p.tiles_per_head = (int)((s.N + 2 * kTile - 1) / (2 * kTile));
   p.n_tiles = p.tiles_per_head * s.Hkv;
   if (p.n_tiles == 0) return cudaSuccess;

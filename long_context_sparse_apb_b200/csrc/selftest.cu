@@ -30,18 +30,6 @@ __global__ void selftest_wait_kernel(DeviceStatus* status, uint64_t short_ns, ui
   }
 }
 
-// Sets the launch-wide abort flag of `status` once delay_ns have passed
-// (one thread), as a CTA whose wait ran out would: every bounded wait of a
-// kernel still running on that status block then gives up at its next
-// unsatisfied check.
-__global__ void abort_after_kernel(DeviceStatus* status, uint64_t delay_ns) {
-  const uint64_t t0 = ptx::globaltimer();
-  while (ptx::globaltimer() - t0 < delay_ns) {
-  }
-  atomicExch(&status->abort, 1u);
-  __threadfence();
-}
-
 }  // namespace
 }  // namespace apb
 
@@ -74,18 +62,4 @@ extern "C" apb_status apb_selftest_wait_timeout(void* workspace, size_t ws_bytes
   const cudaError_t e = apb::launch_wait_selftest(status, limit_us, elapsed,
                                                   reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? APB_OK : apb::cuda_fail(e, "self-test kernel");
-}
-
-extern "C" apb_status apb_selftest_abort_after(void* workspace, size_t ws_bytes, uint32_t delay_us,
-                                               void* stream) {
-  if (!workspace || ws_bytes < apb::kStatusBytes || (reinterpret_cast<uintptr_t>(workspace) & 15))
-    return apb::fail(APB_ERR_INVALID_ARG,
-                     "apb_selftest_abort_after: workspace NULL, unaligned or < %zu bytes",
-                     apb::kStatusBytes);
-  if (delay_us > 1000000)
-    return apb::fail(APB_ERR_INVALID_ARG, "apb_selftest_abort_after: delay_us=%u > 1e6", delay_us);
-  apb::abort_after_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<apb::DeviceStatus*>(workspace), (uint64_t)delay_us * 1000ull);
-  const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? APB_OK : apb::cuda_fail(e, "abort self-test kernel");
 }

@@ -1,6 +1,5 @@
 """Failure detection on the GPU without a fault: a bounded wait that runs out,
-and kernels whose waits are made to give up mid-run through the launch-wide
-abort flag.
+and kernels whose waits are made to run out mid-run by a short wait limit.
 
 apb_selftest_wait_timeout launches two CTAs waiting on barriers that nothing
 completes, through the same bounded-wait primitive and status block as the
@@ -14,9 +13,9 @@ import torch
 
 from long_context_sparse_apb_b200 import inputs
 
-pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.gpu
 def test_wait_timeout_is_reported_and_context_survives():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -44,12 +43,15 @@ def test_wait_timeout_is_reported_and_context_survives():
     assert torch.isfinite(out.float()).all()
 
 
-def test_abort_mid_kernel_is_reported_and_context_survives():
-    """A kernel whose waits start giving up mid-run (the launch-wide abort
-    flag set from another stream, as a CTA whose wait ran out would set it)
-    must still finish -- every warp meets its partners at each remaining
-    named barrier -- and report APB_ERR_TIMEOUT; the context stays usable
-    and the next clean run equals a clean run made before."""
+@pytest.mark.gpu
+@pytest.mark.parametrize("limit_ns", [2_000, 200])
+def test_short_wait_limit_mid_kernel_is_reported_and_context_survives(limit_ns):
+    """With the bounded waits' limit cut to microseconds, the waits that
+    really block (on the tensor core, the copies, the other warps) run out
+    mid-run in the score and attention kernels.  Each call must still finish
+    -- every warp drains and meets its partners at each remaining named
+    barrier -- and report APB_ERR_TIMEOUT; with the limit restored, the next
+    run equals a clean run made before."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from long_context_sparse_apb_b200 import _lib as apb
@@ -63,54 +65,26 @@ def test_abort_mid_kernel_is_reported_and_context_survives():
     ref = run(xd["q"], xd["k"], xd["v"], *w).clone()
     torch.cuda.synchronize()
     assert apb.device_status(run.workspace) == apb.APB_OK
-    side = torch.cuda.Stream()
-
-    # attention (~2 ms at 32K): the one-thread abort kernel fits beside the
-    # attention CTAs and fires 0.5 ms into the launch
     ws = run.workspace
-    ws.zero_()
-    torch.cuda.synchronize()
-    apb.block_attention(c, xd["q"], xd["k"], xd["v"], run.pass_k, run.pass_v, out=run.out,
-                        workspace=ws)
-    apb.selftest_abort_after(ws, 500, stream=side)
-    torch.cuda.synchronize()
-    assert apb.device_status(ws, clear=True) == apb.APB_ERR_TIMEOUT
-
-    ws.zero_()
+    try:
+        apb.selftest_set_wait_limit(limit_ns)
+        apb.block_attention(c, xd["q"], xd["k"], xd["v"], run.pass_k, run.pass_v, out=run.out,
+                            workspace=ws)
+        torch.cuda.synchronize()
+        assert apb.device_status(ws, clear=True) == apb.APB_ERR_TIMEOUT
+        apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, idx=run.idx, workspace=ws)
+        torch.cuda.synchronize()
+        assert apb.device_status(ws, clear=True) == apb.APB_ERR_TIMEOUT
+    finally:
+        apb.selftest_set_wait_limit(0)
     out = run(xd["q"], xd["k"], xd["v"], *w)
     torch.cuda.synchronize()
     assert apb.device_status(ws) == apb.APB_OK
     assert torch.equal(out, ref)
 
 
-def test_abort_mid_score_kernel_is_reported():
-    """The same for the persistent score kernel (128K workload, ~0.5 ms):
-    the abort kernel goes first (it holds one SM, so one CTA pair starts only
-    after it and leaves at once) and fires 0.25 ms later, well after the
-    call's own clearing of the flag and inside the score kernel."""
-    if not torch.cuda.is_available():
-        pytest.skip("no CUDA device")
+def test_wait_limit_argument_checks():
     from long_context_sparse_apb_b200 import _lib as apb
-
-    cfg = inputs.LLAMA8B_128K
-    x = inputs.generate(cfg)
-    xd = {k: v.cuda() for k, v in x.items() if k != "needles"}
-    del x
-    c = apb.make_config(cfg)
-    w = (xd["w1"], xd["b1"], xd["w2"], xd["b2"])
-    ws = apb.new_workspace(c)
-    ref, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, workspace=ws)
-    torch.cuda.synchronize()
-    assert apb.device_status(ws) == apb.APB_OK
-    side = torch.cuda.Stream()
-    ws.zero_()
-    torch.cuda.synchronize()
-    apb.selftest_abort_after(ws, 250, stream=side)
-    apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, workspace=ws)
-    torch.cuda.synchronize()
-    assert apb.device_status(ws, clear=True) == apb.APB_ERR_TIMEOUT
-    ws.zero_()
-    idx, _ = apb.score_compress(c, xd["q"], xd["k"], xd["v"], *w, workspace=ws)
-    torch.cuda.synchronize()
-    assert apb.device_status(ws) == apb.APB_OK
-    assert torch.equal(idx, ref)
+    assert apb._lib.apb_selftest_set_wait_limit(50) == apb.APB_ERR_INVALID_ARG
+    assert "limit_ns=50" in apb._lib.apb_last_error().decode()
+    assert apb._lib.apb_selftest_set_wait_limit(0) == apb.APB_OK
