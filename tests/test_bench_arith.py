@@ -55,3 +55,20 @@ def test_source_rev_ignores_comments_only():
     commented = "// a note\nint f(int x) {  /* why */\n  return x + 1;  // inline\n\n}\n"
     assert bench.source_rev(code) == bench.source_rev(commented)
     assert bench.source_rev(code) != bench.source_rev(code.replace("+ 1", "+ 2"))
+
+
+def test_kv_head_split_shares_the_work_evenly():
+    # the default multi-GPU mode: every rank gets Hkv / N kv heads and their
+    # q heads, so the ranks' attention FLOPs and A1-A3 bytes each are 1/N of
+    # the sequence's (the per-rank roofline uses the rank's share)
+    cfg = inputs.LLAMA8B_128K
+    full_fl = bench.attention_flops(cfg, bench.visible_pairs(cfg))
+    for world in (1, 2, 4, 8):
+        shares = []
+        for rank in range(world):
+            from long_context_sparse_apb_b200.sharded import kv_head_range
+            gb, ge = kv_head_range(cfg.n_kv_heads, rank, world)
+            lcfg = cfg.replace(n_q_heads=(ge - gb) * cfg.group, n_kv_heads=ge - gb)
+            shares.append(bench.attention_flops(lcfg, bench.visible_pairs(lcfg)))
+            assert bench.hbm_bytes_compress(lcfg) * world == bench.hbm_bytes_compress(cfg)
+        assert len(set(shares)) == 1 and abs(sum(shares) - full_fl) < 1.0
