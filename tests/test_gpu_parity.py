@@ -286,11 +286,14 @@ def test_single_call_prefill_equals_three_calls(apb, cfg):
                                  inputs.TINY.replace(n_hosts=5, block_len=300, anchor_len=75,
                                                      keep=130, n_q_heads=10, n_kv_heads=2,
                                                      head_dim=128, seed=13),
-                                 inputs.TINY.replace(keep=512, seed=14)],
-                         ids=["tiny", "ragged_g5", "keep_n"])
+                                 inputs.TINY.replace(keep=512, seed=14),
+                                 inputs.TINY.replace(n_hosts=3, block_len=1000, anchor_len=100,
+                                                     keep=777, seed=15)],
+                         ids=["tiny", "ragged_g5", "keep_n", "ragged_parts"])
 def test_score_compress_pass_equals_separate_calls(apb, cfg):
     # selection and gather in one launch: idx, scores and both passing
-    # buffers equal the two-call path bit for bit
+    # buffers equal the two-call path bit for bit (ragged_parts: the gather
+    # of each (host, kv head) split over 6 CTAs, the last with fewer rows)
     x = inputs.generate(cfg)
     xd = _to_dev(x)
     c = apb.make_config(cfg)
