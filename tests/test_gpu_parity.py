@@ -357,3 +357,14 @@ def test_topk_unstaged_path_large_block(apb):
     assert np.abs(scores.cpu().numpy() - s_ref).max() <= SCORE_ABS
     check_topk(idx.cpu().numpy(), s_ref, cfg)
     _check_passing_exact(x, idx.cpu().numpy(), pk, pv)
+    # the fused form on the same path: each (host, kv head) split over many
+    # CTAs (2 units, 3000 rows), every one re-reading the scores from global
+    # memory; bit-equal to the two calls
+    pk2 = torch.full_like(pk, float("nan"))
+    pv2 = torch.full_like(pv, float("nan"))
+    idx2 = apb.score_compress_pass(c, xd["q"], xd["k"], xd["v"], xd["w1"], xd["b1"], xd["w2"],
+                                   xd["b2"], pk2, pv2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx2, idx)
+    assert torch.equal(pk2.view(torch.int16), pk.view(torch.int16))
+    assert torch.equal(pv2.view(torch.int16), pv.view(torch.int16))
