@@ -157,7 +157,8 @@ __device__ __forceinline__ int chunk_section(int c, int d) { return (c * kChunk)
 // piece ct % 8 (8 features) of every q chunk for the tokens
 // sp * 64 + ct / 8 + 32 i, i < 2, and reads it from the group's G heads, 4
 // heads at a time: the 8 lanes of a token cover a whole 128-byte line per
-// load, and a pass reads each token's G * d * 2 contiguous bytes.  The sums
+// load (streaming loads that skip L1), and a pass reads each token's
+// G * d * 2 contiguous bytes.  The sums
 // run in fp32; the mean (x 1/G) is split into bf16 hi + lo.
 constexpr int kMaxQChunks = 2;             // d <= 128
 
@@ -183,7 +184,7 @@ __device__ __forceinline__ void q_issue(const ScoreParams& p, long long row0, in
         L.v[c][i][u] = make_uint4(0u, 0u, 0u, 0u);
         if (c < n_q && t < p.N && j0 + u < p.G)
           L.v[c][i][u] =
-              __ldg(reinterpret_cast<const uint4*>(base + (long long)u * p.d + c * kChunk));
+              ptx::ld_stream_16(base + (long long)u * p.d + c * kChunk);
       }
   }
 }
